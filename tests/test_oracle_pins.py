@@ -1,0 +1,254 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself:
+closed forms, invariants, brute force on tiny inputs, library routines, and the
+numbers printed in the SAF3R paper.  No GPU is needed."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from saf3r_synth import CORR, DENSE, POSITION, PROBE, SCAN, HeadCfg, Layout
+
+RNG = np.random.default_rng(1234)
+
+
+def small_layout(S=3, g=5, H=2):
+    return Layout(S=S, g=g, H=H)
+
+
+# ---------------------------------------------------------------- attention
+
+def test_single_key_returns_its_value():
+    q = RNG.standard_normal(64)
+    K = RNG.standard_normal((1, 64))
+    V = RNG.standard_normal((1, 64))
+    out = O.attention_rows(q, K, V)[0]
+    assert np.array_equal(out, V[0])
+
+
+def test_two_keys_closed_form_sigmoid():
+    # softmax over two logits a, b is (sigmoid(a-b), sigmoid(b-a)); logits use 1/sqrt(64) = 1/8
+    q = RNG.standard_normal(64)
+    K = RNG.standard_normal((2, 64))
+    V = RNG.standard_normal((2, 64))
+    a, b = float(q @ K[0]) / 8.0, float(q @ K[1]) / 8.0
+    w0 = 1.0 / (1.0 + math.exp(-(a - b)))
+    expect = w0 * V[0] + (1.0 - w0) * V[1]
+    np.testing.assert_allclose(O.attention_rows(q, K, V)[0], expect, rtol=0, atol=1e-13)
+
+
+def test_dense_matches_torch_sdpa_fp64():
+    N = 77
+    Q, K, V = (RNG.standard_normal((N, 64)) for _ in range(3))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None])[0].numpy()
+    np.testing.assert_allclose(O.dense_rows(Q, K, V, np.arange(N)), ref, rtol=0, atol=1e-12)
+
+
+def test_sparse_matches_torch_sdpa_with_mask():
+    # excluded keys behave as logit -inf: the SDPA boolean mask drops them
+    N = 50
+    Q, K, V = (RNG.standard_normal((N, 64)) * 2 for _ in range(3))
+    keep = np.sort(RNG.choice(N, size=17, replace=False))
+    mask = np.zeros((N, N), dtype=bool)
+    mask[:, keep] = True
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None],
+        attn_mask=torch.from_numpy(mask)[None])[0].numpy()
+    np.testing.assert_allclose(O.attention_rows(Q, K[keep], V[keep]), ref, rtol=0, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one_and_identical_keys_are_uniform():
+    q = RNG.standard_normal((5, 64)) * 3
+    K = RNG.standard_normal((40, 64)) * 3
+    w = O.attention_weights(q, K)
+    assert np.all(np.abs(w.sum(axis=1) - 1.0) < 1e-12)
+    Krep = np.repeat(RNG.standard_normal((1, 64)), 9, axis=0)
+    V = RNG.standard_normal((9, 64))
+    np.testing.assert_allclose(O.attention_rows(q, Krep, V), np.repeat(V.mean(0, keepdims=True), 5, 0),
+                               rtol=0, atol=1e-13)
+
+
+def test_kept_set_order_does_not_matter():
+    q = RNG.standard_normal((4, 64))
+    K = RNG.standard_normal((30, 64))
+    V = RNG.standard_normal((30, 64))
+    perm = RNG.permutation(30)
+    np.testing.assert_allclose(O.attention_rows(q, K, V), O.attention_rows(q, K[perm], V[perm]),
+                               rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- Top-K
+
+@pytest.mark.parametrize("k", [1, 3, 7, 20])
+def test_topk_equals_rank_counting_with_ties(k):
+    # many duplicated scores: key j is selected iff fewer than k keys beat it,
+    # where i beats j when s_i > s_j or (s_i == s_j and i < j)
+    s = RNG.integers(0, 5, size=20).astype(np.float32)
+    got = set(O.topk_desc(s, k).tolist())
+    want = set()
+    for j in range(20):
+        beaten = sum(1 for i in range(20) if s[i] > s[j] or (s[i] == s[j] and i < j))
+        if beaten < k:
+            want.add(j)
+    assert got == want
+    ranked = O.topk_desc(s, k)
+    assert all((s[a] > s[b]) or (s[a] == s[b] and a < b) for a, b in zip(ranked, ranked[1:]))
+
+
+def test_probe_equals_column_mean_of_full_score_matrix():
+    # section 4.3: ranking by the column means of QK^T/sqrt(D) equals ranking by
+    # the mean-query probe.  Integer-valued Q, K make every sum exact.
+    L = small_layout(S=2, g=4)
+    Q = RNG.integers(-3, 4, size=(L.N, 64)).astype(np.float32)
+    K = RNG.integers(-3, 4, size=(L.N, 64)).astype(np.float32)
+    full = Q.astype(np.float64) @ K.astype(np.float64).T / 8.0
+    colmean = full.mean(axis=0)
+    patches = O.patch_tokens(L)
+    for k in (1, 5, 11):
+        # brute force ranking of the column means over patch keys
+        order = sorted(patches.tolist(), key=lambda j: (-colmean[j], j))
+        want = np.sort(np.array(order[:k]))
+        got = O.probe_topk(L, O.probe_scores(O.probe_mean(Q), K), k)
+        assert np.array_equal(got, want)
+
+
+def test_probe_set_size_and_specials():
+    L = small_layout()
+    Q = RNG.standard_normal((L.N, 64)).astype(np.float32)
+    K = RNG.standard_normal((L.N, 64)).astype(np.float32)
+    keys = O.probe_topk(L, O.probe_scores(O.probe_mean(Q), K), 13)
+    assert len(keys) == 13 and not O.is_special(L, keys).any()
+    ks = O.probe_set(L, keys)
+    assert len(ks) == 13 + L.n_special * L.S
+
+
+# ---------------------------------------------------------------- static and stride sets
+
+def test_position_set_closed_form_count_and_membership():
+    L = small_layout(S=3, g=5)
+    for i in range(L.N):
+        ks = O.position_set(L, i)
+        s, loc = divmod(i, L.V)
+        base = L.n_special * L.S + L.P
+        if loc < L.n_special:
+            assert len(ks) == base
+        else:
+            r, c = divmod(loc - L.n_special, L.g)
+            nb = (min(r + 1, L.g - 1) - max(r - 1, 0) + 1) * (min(c + 1, L.g - 1) - max(c - 1, 0) + 1)
+            assert len(ks) == base + (L.S - 1) * nb
+        # brute-force membership from the definition
+        want = []
+        for j in range(L.N):
+            sj, lj = divmod(j, L.V)
+            keep = lj < L.n_special or sj == 0
+            if loc >= L.n_special and lj >= L.n_special:
+                r, c = divmod(loc - L.n_special, L.g)
+                rj, cj = divmod(lj - L.n_special, L.g)
+                keep = keep or (abs(rj - r) <= 1 and abs(cj - c) <= 1)
+            if keep:
+                want.append(j)
+        assert np.array_equal(ks, np.array(want))
+
+
+def test_stride_set_closed_form():
+    L = small_layout(S=3, g=5)
+    for s, ph in [(1, 0), (4, 3), (7, 2), (30, 29)]:
+        ks = O.stride_set(L, s, ph)
+        lattice = (L.N - ph + s - 1) // s
+        off = sum(1 for t in O.special_tokens(L) if t % s != ph)
+        assert len(ks) == lattice + off
+        assert all((j % s == ph) or (j % L.V < L.n_special) for j in ks)
+
+
+def test_stride_keep_fraction_matches_paper_table6():
+    rows = [l.split() for l in open("tests/golden/table6_stride_keys.txt") if l.strip() and l[0] != "#"]
+    L = Layout(S=100, g=37, H=1)
+    for stride, pct in rows:
+        s = int(stride)
+        lattice = len(O.stride_set(L, s, 0)) - sum(1 for t in O.special_tokens(L) if t % s != 0)
+        assert round(100.0 * lattice / L.N, 1) == float(pct)
+
+
+# ---------------------------------------------------------------- DINO tiles
+
+def test_tile_cosines_brute_force_and_topk():
+    L = small_layout(S=3, g=7)
+    f = RNG.standard_normal((L.S * L.P, 16)).astype(np.float32) + 0.5
+    means = O.dino_tile_means(L, f)
+    # brute force: explicit loops over tokens and pairs
+    for t in range(L.T):
+        acc, n = np.zeros(16), 0
+        for tok in range(t * 64, min(t * 64 + 64, L.N)):
+            s, loc = divmod(tok, L.V)
+            if loc >= L.n_special:
+                row = f[s * L.P + loc - L.n_special].astype(np.float64)
+                acc += row / math.sqrt(float((row * row).sum()))
+                n += 1
+        np.testing.assert_allclose(means[t], acc / n, rtol=0, atol=1e-14)
+    cos = O.tile_cosines(means)
+    for u in range(L.T):
+        for v in range(L.T):
+            a, b = means[u], means[v]
+            want = float(a @ b) / math.sqrt(float(a @ a) * float(b @ b))
+            assert abs(float(cos[u, v]) - want) <= 1e-6
+    rank = O.tile_topk(cos, L.T)
+    for u in range(L.T):
+        assert sorted(rank[u].tolist()) == list(range(L.T))
+        assert rank[u][0] == u or cos[u, rank[u][0]] >= cos[u, u]
+
+
+def test_corr_set_dedups_specials():
+    L = small_layout(S=3, g=7)
+    tiles = [0, 2]
+    ks = O.corr_set(L, tiles)
+    inside = sum(1 for v in tiles for t in O.tile_tokens(L, v) if t % L.V < L.n_special)
+    assert len(ks) == sum(len(O.tile_tokens(L, v)) for v in tiles) + L.n_special * L.S - inside
+    assert len(set(ks.tolist())) == len(ks)
+
+
+# ---------------------------------------------------------------- reductions to dense
+
+def test_full_budgets_reduce_to_dense():
+    L = small_layout(S=2, g=6)
+    Q, K, V = (RNG.standard_normal((1, L.N, 64)).astype(np.float32) for _ in range(3))
+    dino = RNG.standard_normal((L.S * L.P, 8)).astype(np.float32)
+    rows = np.arange(L.N)
+    dense = O.dense_rows(Q[0], K[0], V[0], rows)
+    for hc in [HeadCfg(PROBE, k=L.S * L.P), HeadCfg(SCAN, stride=1, phase=0), HeadCfg(CORR, k=L.T),
+               HeadCfg(DENSE)]:
+        sel = O.select(L, [hc], Q, K, dino)
+        out = O.sparse_rows(L, hc, sel, 0, Q[0], K[0], V[0], rows)
+        np.testing.assert_allclose(out, dense, rtol=0, atol=1e-12)
+        assert O.nmse(dense, out) < 1e-24
+    L1 = Layout(S=1, g=6, H=1)
+    Q1, K1, V1 = (RNG.standard_normal((L1.N, 64)) for _ in range(3))
+    sel = O.Selection()
+    out = O.sparse_rows(L1, HeadCfg(POSITION), sel, 0, Q1, K1, V1, np.arange(L1.N))
+    np.testing.assert_allclose(out, O.dense_rows(Q1, K1, V1, np.arange(L1.N)), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- NMSE and the profile rule
+
+def test_nmse_closed_forms():
+    a = RNG.standard_normal((10, 64))
+    assert O.nmse(a, a) == 0.0
+    for alpha in (0.0, 0.5, 1.5):
+        assert abs(O.nmse(a, alpha * a) - (1 - alpha) ** 2) < 1e-14
+
+
+def test_choose_config_rule():
+    # cheapest qualifying candidate; ties in cost to the lower index
+    assert O.choose_config([0.5, 0.005, 0.009, 0.001], [10, 40, 30, 30], 1e-2) == 2
+    # nothing qualifies -> least NMSE, ties to the lower index
+    assert O.choose_config([0.5, 0.2, 0.2], [1, 2, 3], 1e-2) == 1
+    assert O.choose_config([0.01, 0.02], [5, 1], 1e-2) == 0
+
+
+def test_kept_pairs_and_omega():
+    L = small_layout(S=2, g=4)
+    sel = O.Selection()
+    pairs = O.kept_pairs(L, HeadCfg(SCAN, stride=3, phase=1), sel, 0)
+    assert pairs == L.N * len(O.stride_set(L, 3, 1))
+    assert O.omega(L, pairs) == 256 * pairs
