@@ -1,0 +1,151 @@
+// Host/device plan structures of the saf3r library (not part of the C ABI).
+#pragma once
+#include <cstdint>
+
+#include "../../include/saf3r.h"
+
+namespace saf3r {
+
+constexpr int kD = 64;            // head dimension
+constexpr int kTile = 64;         // DINO token tile
+constexpr int kMaxHeads = 64;
+constexpr int kItemRows = 256;    // query rows of one attention work item (two 128-row MMA tiles)
+constexpr int kMaxRadius = 3;
+constexpr uint32_t kCacheMagic = 0x52334653u;  // "SF3R"
+constexpr uint32_t kCacheVersion = 1;
+
+// Derived layout numbers.
+struct Dims {
+  int S, gh, gw, ns, H, dino_dim;
+  int P, V, N, T;
+};
+
+inline Dims make_dims(const saf3r_layout& L) {
+  Dims d;
+  d.S = L.S; d.gh = L.grid_h; d.gw = L.grid_w; d.ns = L.n_special; d.H = L.H; d.dino_dim = L.dino_dim;
+  d.P = L.grid_h * L.grid_w;
+  d.V = d.P + L.n_special;
+  d.N = L.S * d.V;
+  d.T = (d.N + kTile - 1) / kTile;
+  return d;
+}
+
+// Cache header (first 256 bytes of the index cache).
+struct CacheHeader {
+  uint32_t magic;
+  uint32_t version;
+  uint64_t hash;            // hash of (layout, cfg)
+  int32_t N, T;
+  int32_t corr_kmax;        // width of the ranked tile list (0 = none)
+  int32_t corr_off;         // int32 offset of the ranked tile list
+  int32_t probe_off[kMaxHeads];  // int32 offset of each probe head's key list (-1 = not a probe head)
+};
+static_assert(sizeof(CacheHeader) <= 512, "cache header too large");
+constexpr int kCacheHeaderBytes = 512;
+
+// A run of key rows of one head, fed to the attention kernel 64 rows at a time.
+// src 0: the caller's K/V ([H][N][64], row = token); src 1: the head's derived
+// rows in the workspace (row relative to the head's derived base).
+struct Seg {
+  int32_t src;
+  int32_t row0;
+  int32_t len;
+  uint32_t flags;   // bits 0-3: member quarters of the 256-row item; bit 4: per-row cell mask;
+                    // bits 8-15 / 16-23: [lo, hi) rows of the run excluded (special tokens inside a tile)
+};
+constexpr uint32_t kSegAllQuarters = 0xFu;
+constexpr uint32_t kSegCellMask = 0x10u;
+
+// Per-head plan of one attention launch (kernel parameter).
+struct HeadPlan {
+  int32_t head;       // head index h in [0, H)
+  int32_t kind;       // saf3r_head_type
+  int32_t q_src;      // 0: caller Q rows are tokens; 1: derived cell-major Q rows (position heads)
+  int32_t q_base;     // derived Q row base (q_src == 1)
+  int32_t kc_base;    // derived K/V row base
+  int32_t n_items;    // work items (256 query rows each)
+  int32_t item_begin; // first global item index
+  int32_t seg_list;   // -1: one implicit segment (below); else Seg offset of item 0's list
+  int32_t seg_cap;    // Seg entries per item
+  int32_t cnt_list;   // offset of the per-item segment counts
+  Seg seg;            // implicit segment
+  int32_t radius;     // position heads
+  int32_t nb_base;    // position heads: derived row where the cell-major neighbour rows start
+};
+
+struct AttnParams {
+  int32_t n_heads;    // entries of heads[] (heads in launch order)
+  int32_t total_items;
+  int32_t S, gh, gw, ns, V, N, P;
+  int32_t out_fp32;
+  void* out;
+  const Seg* segs;
+  const int32_t* seg_counts;
+  int* err;
+  const int* ok_flag;  // nonzero: cache check passed (NULL: no check)
+  long long wait_budget;
+  HeadPlan heads[kMaxHeads];
+};
+
+
+// Selection plan (select.cu).
+struct SelectPlan {
+  int N, V, ns, P, T, dim;
+  int n_probe;
+  int probe_heads[kMaxHeads];
+  int probe_k[kMaxHeads];
+  int probe_off[kMaxHeads];
+  int corr_kmax;
+  int corr_off;
+  CacheHeader header;
+};
+
+// One head's derived-row mapping (prep.cu).
+struct DerivedHead {
+  int head;
+  int kind;
+  int kc_begin;     // first global derived K/V row
+  int n_rows;       // derived K/V rows of this head
+  int qc_begin;     // first global derived Q row (position heads), -1 if none
+  int stride, phase, n_lat;  // scan heads
+  int probe_off;    // cache int32 offset of the probe key list
+  int off_list;     // scan heads: int offset of the off-lattice special list in the workspace
+};
+
+struct DerivedArgs {
+  int n;                    // heads with derived rows
+  int S, V, ns, P, N;
+  long long kc_total;       // derived K/V rows
+  long long qc_total;       // derived Q rows
+  DerivedHead h[kMaxHeads];
+};
+
+}  // namespace saf3r
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace saf3r {
+
+// launchers (each returns the launch error, if any)
+size_t attn_smem_bytes();
+cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, const CUtensorMap& tmQC, const CUtensorMap& tmKC,
+                             const CUtensorMap& tmVC, int num_sms, cudaStream_t stream);
+size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr);
+cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_t* k, const float* dino,
+                          int32_t* cache, uint8_t* ws, cudaStream_t stream, int* n_launch);
+cudaError_t launch_cache_check(const void* cache, uint64_t hash, int N, int T, int* ok, int* err,
+                               cudaStream_t stream);
+cudaError_t launch_derived(const DerivedArgs& a, bool any_scan, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const int32_t* cache, int* offlists, uint16_t* kc, uint16_t* vc,
+                           uint16_t* qc, int* err, int num_sms, cudaStream_t stream, int* n_launch);
+cudaError_t launch_plan_position(int n_items, int S, int gh, int gw, int ns, int N, int R, int cap, Seg* segs,
+                                 int* counts, cudaStream_t stream);
+cudaError_t launch_plan_corr(const int32_t* ranked, int kmax, int kt, int T, int N, int V, int ns, int S,
+                             Seg* segs, int cap, int* counts, int* err, cudaStream_t stream);
+size_t nmse_workspace_bytes(int H);
+cudaError_t launch_nmse(const float* full, const float* sparse, int H, long long per_head, double* part,
+                        double* out, cudaStream_t stream);
+
+}  // namespace saf3r

@@ -1,0 +1,188 @@
+/*
+ * saf3r.h - C ABI of the head-wise dynamic sparse global attention library.
+ *
+ * The method is SAF3R ("SAF3R: Dynamic Sparse Attention for Feed-Forward 3D
+ * Reconstruction Transformers", arXiv 2607.03612).  Every attention head of a
+ * cross-view global-attention layer gets its own key/value index set, chosen
+ * by one of four kernels (section 4.1): a static position/anchor pattern, a
+ * mean-query-probe Top-K (vertical-line heads), a DINO-feature Top-K
+ * (correspondence heads) or a uniform stride (scanning heads).  Exact softmax
+ * attention then runs over the kept keys only; the dynamic sets are built once
+ * per input and cached (section 4.3); an offline step picks each head's
+ * configuration from the output NMSE against full attention (section 4.2).
+ *
+ * Conventions shared by every call
+ *   - Token layout: S views; each view holds n_special special tokens
+ *     (camera, registers) followed by grid_h*grid_w patch tokens in raster
+ *     order.  V = n_special + grid_h*grid_w, N = S*V, token t = s*V + i.
+ *   - Q, K, V, O are row-major [H][N][d] tensors (bf16 inputs; bf16 or fp32
+ *     output), d = 64, rows of 128 bytes.  DINO features are fp32
+ *     [S*grid_h*grid_w][dino_dim], one row per patch token in token order.
+ *   - All pointers named q, k, v, dino, out, cache and workspace are DEVICE
+ *     pointers, 16-byte aligned.  `stream` is a cudaStream_t (NULL = legacy
+ *     default stream).  The caller owns every buffer; the library allocates
+ *     no device memory and keeps no state except one error word per device.
+ *   - Calls are asynchronous on `stream` unless stated.  Argument errors are
+ *     returned at once and launch nothing.  Errors found on the device (a
+ *     bounded wait that expired, an index cache built for another layout)
+ *     are recorded in the device error word and reported by saf3r_check().
+ *   - Attention scale is 1/sqrt(d); excluded keys take no part in the softmax
+ *     (their logit is -inf), so each row is an exact softmax over its kept set.
+ */
+#ifndef SAF3R_H
+#define SAF3R_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SAF3R_OK = 0,
+    SAF3R_ERR_INVALID = 1,      /* bad argument, or cache/layout mismatch found on the device */
+    SAF3R_ERR_CUDA = 2,         /* a CUDA runtime/driver call failed */
+    SAF3R_ERR_TIMEOUT = 3,      /* a bounded device wait expired; the kernel gave up cleanly */
+    SAF3R_ERR_INDEX = 4,        /* an index read from the cache was out of range */
+    SAF3R_ERR_UNSUPPORTED = 5   /* shape or device not supported (d != 64, not sm_100) */
+} saf3r_status;
+
+/* Head kinds (section 3, Observation #2; kernels of section 4.1). */
+typedef enum {
+    SAF3R_POSITION = 0,  /* static kernel: specials + anchor view 0 + the 3x3 cell neighbourhood in every view */
+    SAF3R_PROBE = 1,     /* query-probe Top-K: Top-k patch keys by mean-query score, + all specials */
+    SAF3R_CORR = 2,      /* DINO Top-K, block-wise: per 64-query tile, Top-k 64-token key tiles + all specials */
+    SAF3R_SCAN = 3,      /* uniform sampling: keys j with j mod stride == phase, + all specials */
+    SAF3R_DENSE = 4      /* every key (full attention) */
+} saf3r_head_type;
+
+typedef struct {
+    int32_t S;          /* views, >= 1 */
+    int32_t grid_h;     /* patch rows per view */
+    int32_t grid_w;     /* patch columns per view */
+    int32_t n_special;  /* special tokens per view (5: 1 camera + 4 registers) */
+    int32_t H;          /* heads, 1..64 */
+    int32_t d;          /* head dimension; must be 64 */
+    int32_t dino_dim;   /* DINO feature width (384); 1..1024 */
+    int32_t tile;       /* token tile of the block-wise DINO kernel; must be 64 */
+} saf3r_layout;
+
+typedef struct {
+    int32_t type;       /* saf3r_head_type */
+    int32_t k;          /* PROBE: kept patch keys (1..S*grid_h*grid_w); CORR: kept key tiles (1..T) */
+    int32_t stride;     /* SCAN: >= 1 */
+    int32_t phase;      /* SCAN: 0 <= phase < stride */
+    int32_t radius;     /* POSITION: neighbourhood radius in cells, 0..3 (1 = 3x3) */
+} saf3r_head_cfg;
+
+/* Operations for saf3r_workspace_bytes. */
+enum { SAF3R_OP_SELECT = 0, SAF3R_OP_SPARSE = 1, SAF3R_OP_DENSE = 2, SAF3R_OP_PROFILE = 3 };
+
+/*
+ * Size in bytes of the index cache that saf3r_select_kv fills for this layout
+ * and per-head configuration (cfg: H entries).  The cache holds a header with
+ * a hash of (layout, cfg), each probe head's kept patch keys (int32, ascending)
+ * and, if any head is CORR, the ranked key-tile list of every query tile
+ * (int32 [T][kmax], best first; T = ceil(N/64), kmax = largest CORR k).
+ * Returns 0 for an invalid layout or cfg.
+ */
+size_t saf3r_cache_bytes(const saf3r_layout* layout, const saf3r_head_cfg* cfg);
+
+/*
+ * Size in bytes of the device workspace that operation `op` needs:
+ * SAF3R_OP_SELECT or SAF3R_OP_SPARSE with the per-head cfg (H entries),
+ * SAF3R_OP_DENSE with cfg = NULL.  Profiling uses
+ * saf3r_profile_workspace_bytes.  Returns 0 for invalid arguments.
+ */
+size_t saf3r_workspace_bytes(const saf3r_layout* layout, const saf3r_head_cfg* cfg, int op);
+
+/* Workspace bytes of saf3r_profile_heads for n_cand candidates. */
+size_t saf3r_profile_workspace_bytes(const saf3r_layout* layout, const saf3r_head_cfg* cand, int n_cand);
+
+/*
+ * Build the per-input dynamic index sets (section 4.3, "Online Pattern
+ * Adaptation") and write them to `cache` (saf3r_cache_bytes bytes).
+ *   - PROBE heads: qbar = mean of all N query rows of the head (fp64 sum,
+ *     rounded once to fp32); score_j = qbar . k_j / sqrt(d) in fp32; the k
+ *     patch keys of highest score (ties to the lower token index) are kept.
+ *     Section 4.3 shows this ranking equals ranking keys by the column means
+ *     of Q K^T / sqrt(d).
+ *   - CORR heads: each flat 64-token tile gets the mean of the L2-normalised
+ *     DINO features of its patch tokens; tiles are compared by cosine; every
+ *     query tile ranks all tiles (itself included; ties to the lower tile).
+ *     Computed once and shared by all CORR heads (prefixes serve smaller k).
+ *   - POSITION, SCAN and DENSE heads need no cached state.
+ * q, k: bf16 [H][N][d]; dino: fp32 patch features, or NULL when no head is CORR.
+ * workspace: saf3r_workspace_bytes(layout, cfg, SAF3R_OP_SELECT) bytes.
+ */
+saf3r_status saf3r_select_kv(const saf3r_layout* layout, const saf3r_head_cfg* cfg,
+                             const void* q, const void* k, const float* dino,
+                             void* cache, void* workspace, void* stream);
+
+/*
+ * Sparse global attention over cached index sets (section 4.1): for every head
+ * h and query i, O[h][i] = sum_{j in kept(h,i)} softmax_j(q.k_j/sqrt(d)) v_j.
+ * `cache` must come from saf3r_select_kv with the same layout and cfg (checked
+ * on the device through the cache header hash; a mismatch records
+ * SAF3R_ERR_INVALID and leaves `out` unwritten).  q, k, v may be fresh
+ * tensors of a later layer call: the cached sets are reused as they are.
+ * out: bf16 [H][N][d] (out_is_fp32 = 0) or fp32 (out_is_fp32 = 1).
+ * workspace: saf3r_workspace_bytes(layout, cfg, SAF3R_OP_SPARSE) bytes.
+ */
+saf3r_status saf3r_sparse_attn(const saf3r_layout* layout, const saf3r_head_cfg* cfg, const void* cache,
+                               const void* q, const void* k, const void* v,
+                               void* out, int out_is_fp32, void* workspace, void* stream);
+
+/*
+ * Full attention over all N keys for every head: O_full of section 4.2, the
+ * reference of the per-head NMSE.  Layout arguments as saf3r_sparse_attn.
+ * workspace: saf3r_workspace_bytes(layout, NULL, SAF3R_OP_DENSE) bytes.
+ */
+saf3r_status saf3r_dense_attn(const saf3r_layout* layout, const void* q, const void* k, const void* v,
+                              void* out, int out_is_fp32, void* workspace, void* stream);
+
+/*
+ * Offline head profiling (section 4.2) on one calibration input.  For every
+ * candidate c (n_cand entries; a SCAN candidate's phase is replaced by
+ * head mod stride) and every head h it computes
+ *     nmse[h*n_cand + c]  = ||O_full - O_c||^2 / ||O_full||^2        (eq. 1)
+ *     pairs[h*n_cand + c] = number of (query, kept key) pairs (Omega = 4*d*pairs)
+ * and chooses for each head the candidate of least Omega whose NMSE is at
+ * most nmse_max (ties to the lower candidate index); when none qualifies, the
+ * candidate of least NMSE (the argmin of eq. 2).  chosen (H entries), nmse
+ * and pairs are HOST arrays.  Synchronizes `stream`.
+ * workspace: saf3r_profile_workspace_bytes(layout, cand, n_cand) bytes.
+ */
+saf3r_status saf3r_profile_heads(const saf3r_layout* layout, const saf3r_head_cfg* cand, int n_cand,
+                                 const void* q, const void* k, const void* v, const float* dino,
+                                 double nmse_max, saf3r_head_cfg* chosen, double* nmse, int64_t* pairs,
+                                 void* workspace, void* stream);
+
+/*
+ * Copy one head's cached index list to host memory (synchronizes `stream`):
+ * PROBE head -> its k kept patch keys (ascending); CORR head -> the ranked
+ * tile list int32 [T][k] truncated to that head's k.  *n receives the number
+ * of entries; at most `cap` are written.  Other head kinds return
+ * SAF3R_ERR_INVALID.
+ */
+saf3r_status saf3r_cache_export(const saf3r_layout* layout, const saf3r_head_cfg* cfg, const void* cache,
+                                int head, int32_t* host_idx, size_t cap, size_t* n, void* stream);
+
+/*
+ * Synchronize `stream`, then read and clear the calling device's error word.
+ * Returns SAF3R_OK or the first device-side error recorded since the last check.
+ */
+saf3r_status saf3r_check(void* stream);
+
+/* Number of kernels the last saf3r_* call on this host thread launched. */
+int saf3r_last_launch_count(void);
+
+/* Static text for a status code. */
+const char* saf3r_status_string(saf3r_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAF3R_H */

@@ -1,0 +1,53 @@
+"""Comparison helpers of the GPU parity tests (test code only)."""
+import numpy as np
+
+import oracle as O
+
+# tolerances of the GPU path against the oracle (bf16 inputs, fp32 accumulation)
+MAX_ABS = 1e-2
+REL_L2 = 5e-3
+BOUNDARY_REL = 1e-5
+
+
+def compare_outputs(gpu: np.ndarray, ref: np.ndarray, what: str):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(gpu).all(), f"{what}: non-finite output"
+    err = np.abs(gpu - ref)
+    rel = np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert err.max() <= MAX_ABS, f"{what}: max-abs {err.max():.3e} > {MAX_ABS}"
+    assert rel <= REL_L2, f"{what}: rel-L2 {rel:.3e} > {REL_L2}"
+    return float(err.max()), float(rel)
+
+
+def check_topk_set(gpu_keys, ref_ranked, scores, k, what):
+    """gpu_keys: the GPU's kept set; ref_ranked: the oracle's candidates in rank order
+    (at least k); scores: oracle fp32 score per candidate id.  The sets must agree
+    except for keys whose score is within BOUNDARY_REL of the k-th score.
+    Returns True when the sets are identical."""
+    g = set(int(x) for x in np.asarray(gpu_keys).tolist())
+    r = set(int(x) for x in np.asarray(ref_ranked[:k]).tolist())
+    assert len(g) == k, f"{what}: {len(g)} distinct keys, expected {k}"
+    if g == r:
+        return True
+    kth = float(scores[int(ref_ranked[k - 1])])
+    tol = BOUNDARY_REL * max(abs(kth), 1e-30)
+    for x in g ^ r:
+        assert abs(float(scores[x]) - kth) <= tol, \
+            f"{what}: key {x} score {float(scores[x])!r} vs k-th {kth!r} outside the boundary band"
+    return False
+
+
+def check_probe(gpu_keys, L, sel, h, k, what):
+    ranked = O.topk_desc(sel.probe_scores[h], k + 8, O.patch_tokens(L))
+    return check_topk_set(gpu_keys, ranked, sel.probe_scores[h], k, what)
+
+
+def check_tiles(gpu_ranked, sel, k, what):
+    """gpu_ranked: int [T][k] from the cache export."""
+    T = sel.tile_cos.shape[0]
+    exact = True
+    for u in range(T):
+        ranked = O.topk_desc(sel.tile_cos[u], min(T, k + 8))
+        exact &= check_topk_set(gpu_ranked[u], ranked, sel.tile_cos[u], k, f"{what} tile {u}")
+    return exact

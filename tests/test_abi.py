@@ -1,0 +1,67 @@
+"""The C-ABI library loads, exports every symbol include/saf3r.h declares, and
+rejects bad arguments on the host (no GPU needed: no compute call is made)."""
+import ctypes
+
+import pytest
+
+import head_wise_dynamic_b200 as hw
+from saf3r_synth import WORKLOADS
+
+
+def test_library_exports_every_declared_symbol():
+    names = hw.header_functions()
+    assert "saf3r_select_kv" in names and "saf3r_sparse_attn" in names
+    L = hw.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    for s in range(6):
+        assert hw.status_string(s)
+
+
+def _tiny():
+    wl = WORKLOADS["tiny"]
+    return hw.layout_of(wl.layout), hw.cfg_array(wl.heads)
+
+
+def test_sizes_on_host():
+    L, cfg = _tiny()
+    cb = hw.saf3r_cache_bytes(L, cfg)
+    # header (512 B) + 128 probe keys + T*kmax corr tiles (T = 17, kmax = 4)
+    assert cb >= 512 + 128 * 4 + 17 * 4 * 4
+    assert hw.saf3r_workspace_bytes(L, cfg, hw.OP_SELECT) > 0
+    assert hw.saf3r_workspace_bytes(L, cfg, hw.OP_SPARSE) > 0
+    assert hw.saf3r_workspace_bytes(L, None, hw.OP_DENSE) > 0
+
+
+@pytest.mark.parametrize("field,value", [("d", 128), ("tile", 32), ("H", 0), ("H", 65), ("S", 0),
+                                         ("n_special", 64), ("dino_dim", 6)])
+def test_bad_layout_sizes_zero(field, value):
+    L, cfg = _tiny()
+    setattr(L, field, value)
+    assert hw.saf3r_cache_bytes(L, cfg) == 0
+
+
+@pytest.mark.parametrize("h,field,value", [(1, "k", 0), (1, "k", 10 ** 6), (2, "k", 18), (3, "stride", 0),
+                                           (3, "phase", 8), (0, "radius", 4), (0, "type", 9)])
+def test_bad_cfg_sizes_zero(h, field, value):
+    L, cfg = _tiny()
+    setattr(cfg[h], field, value)
+    assert hw.saf3r_cache_bytes(L, cfg) == 0
+
+
+def test_calls_reject_bad_arguments_before_any_launch():
+    L, cfg = _tiny()
+    lib = hw.lib()
+    # null device pointers
+    assert lib.saf3r_select_kv(ctypes.byref(L), cfg, None, None, None, None, None, None) == hw.ERR_INVALID
+    assert lib.saf3r_sparse_attn(ctypes.byref(L), cfg, None, None, None, None, None, 0, None, None) == hw.ERR_INVALID
+    # misaligned pointers
+    bad = 0x1008
+    assert lib.saf3r_dense_attn(ctypes.byref(L), bad, bad, bad, bad, 0, bad, None) == hw.ERR_INVALID
+    # head dimension other than 64 is unsupported
+    L.d = 128
+    assert lib.saf3r_dense_attn(ctypes.byref(L), 0x1000, 0x1000, 0x1000, 0x1000, 0, 0x1000, None) == \
+        hw.ERR_UNSUPPORTED
