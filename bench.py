@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the head-wise dynamic sparse global-attention hot path.
+
+One step = one pass of the whole path over one input of the S=100-view layer:
+the per-input index build (saf3r_select_kv: probe Top-K for 4 heads, DINO
+tile Top-K shared by 4 heads) followed by 4 layer calls of saf3r_sparse_attn
+that reuse the cached indices with fresh Q/K/V.  `value` is kept-pair TFLOP/s
+(256 FLOP per (query, kept key) pair, d = 64) of the whole step, inputs
+resident in HBM; `e2e` is the same metric through the same public API with
+the step's inputs copied from pinned host memory and its outputs copied back.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun); the path does not shard, so each
+rank runs an independent replica and `value` sums the ranks' work over the
+slowest rank's time.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "global-attn layer ms & kept-pair TFLOP/s (% bf16 peak), S=100 views"
+FLOP_PER_PAIR = 256  # q.k (2d) + p.v (2d), d = 64
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_desc(wl):
+    from saf3r_synth import KIND_NAMES
+    L = wl.layout
+    kinds = []
+    for h, hc in enumerate(wl.heads):
+        p = {1: f" Top-{hc.k}", 2: f" tile Top-{hc.k}", 3: f" stride {hc.stride}"}.get(hc.kind, "")
+        kinds.append(f"{h}:{KIND_NAMES[hc.kind]}{p}")
+    return (f"{wl.name}: S={L.S} views x ({L.g}x{L.g} patches + {L.n_special} special) = {L.N} tokens, "
+            f"H={L.H}, d={L.d}; heads [{', '.join(kinds)}]; one index build + {wl.calls} layer calls "
+            f"reusing the cache")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (clock, power, throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+
+        sm = [num(r[1]) for r in rows]
+        mx = max(num(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s in sm if s == s and s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(num(r[3]) for r in rows)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import head_wise_dynamic_b200 as hw
+    from saf3r_synth import WORKLOADS, Scene, qkv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    wl = WORKLOADS[args.workload]
+    L = wl.layout
+    scene = Scene(wl)
+    calls = [qkv(scene, c, device=dev) for c in range(wl.calls)]
+    dino = torch.from_numpy(scene.dino()).to(dev)
+    att = hw.SparseGlobalAttention(L, wl.heads, device=dev)
+    outs = [torch.empty_like(calls[0][0]) for _ in range(wl.calls)]
+    stream = torch.cuda.current_stream(dev)
+
+    # kept pairs of one layer call (exact, from the cache) and the dense reference time
+    att.select(calls[0][0], calls[0][1], dino)
+    pairs = hw.saf3r_kept_pairs(att.layout, att.cfg, att.cache)
+    pairs_call = int(pairs.sum())
+    flops_step = wl.calls * pairs_call * FLOP_PER_PAIR
+
+    n_ev = args.steps * wl.calls
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+    ev_call = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+    ev_sel = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    launches = {"n": 0}
+
+    def step(i=None):
+        if i is not None:
+            ev_sel[i][0].record(stream)
+        att.select(calls[0][0], calls[0][1], dino)
+        launches["n"] += hw.saf3r_last_launch_count()
+        if i is not None:
+            ev_sel[i][1].record(stream)
+        for c in range(wl.calls):
+            if i is not None:
+                e = ev[i * wl.calls + c]
+                hw.saf3r_set_kernel_events(e[0], e[1])
+                ev_call[i * wl.calls + c][0].record(stream)
+            att(calls[c][0], calls[c][1], calls[c][2], out=outs[c])
+            launches["n"] += hw.saf3r_last_launch_count()
+            if i is not None:
+                ev_call[i * wl.calls + c][1].record(stream)
+        hw.saf3r_set_kernel_events(None, None)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    hw.saf3r_check()
+    launches_per_step = launches["n"] // max(args.warmup, 1)
+
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    hw.saf3r_check()
+    ms_step = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms_step], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step = float(tt.item())
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    call_ms = [a.elapsed_time(b) for a, b in ev_call]
+    sel_ms = [a.elapsed_time(b) for a, b in ev_sel]
+    attn_kernel_ms = statistics.mean(kern_ms)
+
+    # dense attention on the same inputs (the library's own dense kernel)
+    out_d = torch.empty_like(outs[0])
+    wsd = torch.empty(hw.saf3r_workspace_bytes(att.layout, None, hw.OP_DENSE), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        hw.saf3r_dense_attn(att.layout, calls[0][0], calls[0][1], calls[0][2], out_d, wsd)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(3):
+        hw.saf3r_dense_attn(att.layout, calls[0][0], calls[0][1], calls[0][2], out_d, wsd)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    hw.saf3r_check()
+    dense_ms = d0.elapsed_time(d1) / 3
+    dense_flops = L.H * L.N * L.N * FLOP_PER_PAIR
+    del out_d
+
+    peaks, peak_src = load_peaks()
+    timed_s = ms_step * args.steps / 1e3
+    peak_key = "bf16_tflops_sustained" if timed_s > 1.0 else "bf16_tflops"
+    peak = float(peaks[peak_key])
+    achieved = pairs_call * FLOP_PER_PAIR / (attn_kernel_ms * 1e-3) / 1e12
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+
+    # end to end through the same API: pinned host inputs in, outputs back, every step
+    e2e = None
+    if not args.no_e2e:
+        host_in = [[t.to("cpu").pin_memory() for t in c] for c in calls]
+        dino_h = dino.to("cpu").pin_memory()
+        host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        h2d = sum(t.numel() * t.element_size() for c in host_in for t in c) + dino_h.numel() * 4
+        d2h = sum(o.numel() * o.element_size() for o in host_out)
+
+        def e2e_step():
+            for c in range(wl.calls):
+                for j in range(3):
+                    calls[c][j].copy_(host_in[c][j], non_blocking=True)
+            dino.copy_(dino_h, non_blocking=True)
+            step()
+            for c in range(wl.calls):
+                host_out[c].copy_(outs[c], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        hw.saf3r_check()
+        e2e_ms = a.elapsed_time(b) / args.e2e_steps
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, scene, calls[0], pairs_call, budget_s=args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "l2": "inputs larger than L2 (Q/K/V 3 x 281 MB per call)",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "layer_ms": ms_step / wl.calls,
+        "attn_call_ms": statistics.mean(call_ms),
+        "attn_kernel_ms": attn_kernel_ms,
+        "select_ms": statistics.mean(sel_ms),
+        "kept_pairs_per_call": pairs_call,
+        "kept_pair_tflops_attn_kernel": achieved,
+        "pct_bf16_peak_attn_kernel": 100.0 * achieved / peak,
+        "dense_ms": dense_ms, "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+        "speedup_vs_dense": dense_ms / statistics.mean(call_ms),
+        "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} {peak_key}",
+                     "algorithmic": f"{pairs_call} kept pairs x 256 FLOP per launch"},
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clock_info,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(wl, scene, qkv_call, pairs_call, budget_s=15.0, rows_per_head=None):
+    """The oracle, as it stands, on a bounded sample of the same workload.
+
+    Times the full index selection of one input and the sparse attention of a
+    few sampled rows per head, then extrapolates the rows to all N rows of the
+    4 layer calls: value = 4 * pairs * 256 / (t_select + 4 * t_rows * pairs / sampled_pairs)."""
+    import oracle as O
+    from saf3r_synth import bf16_to_f32, sample_rows
+
+    L = wl.layout
+    Q, K, V = (bf16_to_f32(t) for t in qkv_call)
+    dino = scene.dino()
+    t = time.perf_counter()
+    sel = O.select(L, wl.heads, Q, K, dino)
+    t_sel = time.perf_counter() - t
+    rows_per_head = rows_per_head or 16
+    sampled_pairs = 0
+    t_rows = 0.0
+    for h, hc in enumerate(wl.heads):
+        rows = sample_rows(wl, h, rows_per_head, seed_extra=1)[:rows_per_head]
+        t = time.perf_counter()
+        O.sparse_rows(L, hc, sel, h, Q[h], K[h], V[h], rows)
+        t_rows += time.perf_counter() - t
+        sampled_pairs += sum(O.kept_count(L, hc, sel, h, int(i)) for i in rows)
+    t_step = t_sel + wl.calls * t_rows * (pairs_call / sampled_pairs)
+    return {"value": wl.calls * pairs_call * FLOP_PER_PAIR / t_step / 1e12, "unit": "TFLOP/s",
+            "cores": _blas_threads(), "kind": "oracle",
+            "sample": (f"full index selection of one input ({t_sel:.1f} s) + sparse attention of "
+                       f"{rows_per_head} sampled rows per head ({t_rows:.2f} s, {sampled_pairs} kept pairs), "
+                       f"extrapolated to all {L.N} rows x {L.H} heads x {wl.calls} calls"),
+            "seconds": t_sel + t_rows}
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    from saf3r_synth import WORKLOADS, Scene, qkv
+
+    wl = WORKLOADS[args.workload]
+    scene = Scene(wl)
+    calls = qkv(scene, 0, device="cpu")
+    # exact kept pairs of one call from the oracle's own selection
+    import oracle as O
+    from saf3r_synth import bf16_to_f32
+    Q, K = bf16_to_f32(calls[0]), bf16_to_f32(calls[1])
+    sel = O.select(wl.layout, wl.heads, Q, K, scene.dino())
+    pairs_call = sum(O.kept_pairs(wl.layout, hc, sel, h) for h, hc in enumerate(wl.heads))
+    vals, secs = [], []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(wl, scene, calls, pairs_call, rows_per_head=4)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            secs.append(r["seconds"])
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "parallelism": "single"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    del torch
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="s100")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -74,6 +74,10 @@ def lib() -> ctypes.CDLL:
         L.saf3r_cache_export.argtypes = [LP, CP, vp, i32, ctypes.POINTER(ctypes.c_int32), sz,
                                          ctypes.POINTER(ctypes.c_size_t), vp]
         L.saf3r_cache_export.restype = i32
+        L.saf3r_kept_pairs.argtypes = [LP, CP, vp, ctypes.POINTER(ctypes.c_int64), vp]
+        L.saf3r_kept_pairs.restype = i32
+        L.saf3r_set_kernel_events.argtypes = [vp, vp]
+        L.saf3r_set_kernel_events.restype = None
         L.saf3r_check.argtypes = [vp]
         L.saf3r_check.restype = i32
         L.saf3r_last_launch_count.argtypes = []
@@ -214,6 +218,21 @@ def saf3r_cache_export(layout, cfg, cache, head: int, stream=None) -> np.ndarray
                                   _stream(stream))
     _check(st, "saf3r_cache_export")
     return out
+
+
+def saf3r_kept_pairs(layout, cfg, cache, stream=None) -> np.ndarray:
+    L = layout_of(layout)
+    out = np.zeros(L.H, dtype=np.int64)
+    st = lib().saf3r_kept_pairs(ctypes.byref(L), _cfg(cfg), _ptr(cache),
+                                out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), _stream(stream))
+    _check(st, "saf3r_kept_pairs")
+    return out
+
+
+def saf3r_set_kernel_events(start=None, stop=None):
+    """Record torch.cuda.Event pair around the attention kernel of following calls (None, None: off)."""
+    lib().saf3r_set_kernel_events(None if start is None else start.cuda_event,
+                                  None if stop is None else stop.cuda_event)
 
 
 def saf3r_check(stream=None):

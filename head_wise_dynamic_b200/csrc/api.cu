@@ -21,6 +21,7 @@ namespace {
 __device__ int g_device_error;  // the one piece of library state: first device-side error since the last check
 
 thread_local int t_launches = 0;
+thread_local cudaEvent_t t_ev_start = nullptr, t_ev_stop = nullptr;
 
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (~2 s) before a device wait gives up
 
@@ -451,8 +452,11 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
       !make_map_2d(&tvc, vc_base, s.kc_rows > 0 ? s.kc_rows : 1) ||
       !make_map_2d(&tqc, qc_base, s.qc_rows > 0 ? s.qc_rows : 1))
     return SAF3R_ERR_CUDA;
+  if (t_ev_start && t_ev_stop && cudaEventRecord(t_ev_start, stream) != cudaSuccess) return SAF3R_ERR_CUDA;
   st = cuda_status(launch_attention(p, tq, tk, tv, tqc, tkc, tvc, dev.sms, stream));
   ++launches;
+  if (st == SAF3R_OK && t_ev_start && t_ev_stop && cudaEventRecord(t_ev_stop, stream) != cudaSuccess)
+    return SAF3R_ERR_CUDA;
   t_launches += launches;
   return st;
 }
@@ -475,6 +479,11 @@ const char* saf3r_status_string(saf3r_status s) {
 }
 
 int saf3r_last_launch_count(void) { return t_launches; }
+
+void saf3r_set_kernel_events(void* start, void* stop) {
+  t_ev_start = static_cast<cudaEvent_t>(start);
+  t_ev_stop = static_cast<cudaEvent_t>(stop);
+}
 
 size_t saf3r_cache_bytes(const saf3r_layout* L, const saf3r_head_cfg* cfg) {
   if (check_layout(L) != SAF3R_OK) return 0;
@@ -687,6 +696,28 @@ static long long pairs_of(const Dims& d, const saf3r_head_cfg& c, const std::vec
     }
   }
   return 0;
+}
+
+saf3r_status saf3r_kept_pairs(const saf3r_layout* L, const saf3r_head_cfg* cfg, const void* cache, int64_t* pairs,
+                              void* stream) {
+  saf3r_status st = check_layout(L);
+  if (st != SAF3R_OK) return st;
+  const Dims d = make_dims(*L);
+  if ((st = check_cfg(d, cfg, L->H)) != SAF3R_OK) return st;
+  if (!pairs) return SAF3R_ERR_INVALID;
+  const CacheLayout cl = cache_layout(d, cfg);
+  std::vector<int32_t> ranked;
+  if (cl.corr_kmax > 0) {
+    if (!cache) return SAF3R_ERR_INVALID;
+    ranked.resize(static_cast<size_t>(d.T) * cl.corr_kmax);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(ranked.data(), static_cast<const int32_t*>(cache) + cl.corr_off, ranked.size() * 4,
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return SAF3R_ERR_CUDA;
+  }
+  for (int h = 0; h < d.H; ++h) pairs[h] = pairs_of(d, cfg[h], ranked, cl.corr_kmax);
+  return SAF3R_OK;
 }
 
 saf3r_status saf3r_profile_heads(const saf3r_layout* L, const saf3r_head_cfg* cand, int n_cand, const void* q,

@@ -170,6 +170,24 @@ saf3r_status saf3r_cache_export(const saf3r_layout* layout, const saf3r_head_cfg
                                 int head, int32_t* host_idx, size_t cap, size_t* n, void* stream);
 
 /*
+ * Exact number of (query, kept key) pairs of every head under (layout, cfg)
+ * with the index sets held in `cache` (section 4.2: the cost of a
+ * configuration is Omega = 4*d*pairs FLOPs).  pairs: HOST int64 [H].
+ * Synchronizes `stream` (the correspondence heads' tile lists are read back).
+ */
+saf3r_status saf3r_kept_pairs(const saf3r_layout* layout, const saf3r_head_cfg* cfg, const void* cache,
+                              int64_t* pairs, void* stream);
+
+/*
+ * Timing hook for measurement: when start and stop are both non-NULL
+ * cudaEvent_t handles, every following saf3r_sparse_attn / saf3r_dense_attn
+ * call made on this host thread records `start` on its stream right before
+ * its attention kernel and `stop` right after it.  NULL, NULL switches the
+ * hook off.  The events are owned by the caller.
+ */
+void saf3r_set_kernel_events(void* start, void* stop);
+
+/*
  * Synchronize `stream`, then read and clear the calling device's error word.
  * Returns SAF3R_OK or the first device-side error recorded since the last check.
  */
