@@ -150,6 +150,9 @@ def run_ours(args):
     ev_call = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
     ev_sel = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+    for a, b in ev:  # torch creates CUDA events lazily: record once so the handles exist
+        a.record(stream)
+        b.record(stream)
     launches = {"n": 0}
 
     def step(i=None):

@@ -230,7 +230,9 @@ def saf3r_kept_pairs(layout, cfg, cache, stream=None) -> np.ndarray:
 
 
 def saf3r_set_kernel_events(start=None, stop=None):
-    """Record torch.cuda.Event pair around the attention kernel of following calls (None, None: off)."""
+    """Record torch.cuda.Event pair around the attention kernel of following calls (None, None: off).
+
+    torch creates CUDA events lazily: record each event once before handing it over."""
     lib().saf3r_set_kernel_events(None if start is None else start.cuda_event,
                                   None if stop is None else stop.cuda_event)
 
