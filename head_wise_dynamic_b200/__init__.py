@@ -16,7 +16,8 @@ from typing import List, Optional, Sequence
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsaf3r.so")
+# SAF3R_LIB may point at another build of the same library (e.g. a debug build).
+LIB_PATH = os.environ.get("SAF3R_LIB") or os.path.join(_HERE, "libsaf3r.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "saf3r.h")
 
 # saf3r_status

@@ -172,6 +172,7 @@ struct CacheLayout {
   int probe_off[kMaxHeads];
   int corr_off = 0;
   int corr_kmax = 0;
+  int order_off = 0;
   size_t bytes = 0;
 };
 
@@ -188,6 +189,8 @@ CacheLayout cache_layout(const Dims& d, const saf3r_head_cfg* cfg) {
   }
   c.corr_off = static_cast<int>(ints);
   ints += static_cast<size_t>(d.T) * c.corr_kmax;
+  c.order_off = static_cast<int>(ints);
+  if (c.corr_kmax > 0) ints += static_cast<size_t>(d.T);
   c.bytes = align256(ints * 4);
   return c;
 }
@@ -382,8 +385,9 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
       st = cuda_status(launch_plan_position(l.n_items, d.S, d.gh, d.gw, d.ns, d.N, l.param, l.cap,
                                             segs + l.seg_begin, cnts + l.cnt_begin, stream));
     } else {
-      st = cuda_status(launch_plan_corr(cache_i + cl.corr_off, cl.corr_kmax, l.param, d.T, d.N, d.V, d.ns, d.S,
-                                        segs + l.seg_begin, l.cap, cnts + l.cnt_begin, dev.err, stream));
+      st = cuda_status(launch_plan_corr(cache_i + cl.corr_off, cache_i + cl.order_off, cl.corr_kmax, l.param, d.T,
+                                        d.N, d.V, d.ns, d.S, segs + l.seg_begin, l.cap, cnts + l.cnt_begin, dev.err,
+                                        stream));
     }
     ++launches;
     if (st != SAF3R_OK) return st;
@@ -403,8 +407,8 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     HeadPlan& hp = p.heads[i];
     hp.head = h;
     hp.kind = c.type;
-    hp.q_src = c.type == SAF3R_POSITION ? 1 : 0;
-    hp.q_base = s.qc_begin[h] < 0 ? 0 : s.qc_begin[h];
+    hp.q_src = c.type == SAF3R_POSITION ? 1 : (c.type == SAF3R_CORR ? 2 : 0);
+    hp.q_base = c.type == SAF3R_CORR ? cl.order_off : (s.qc_begin[h] < 0 ? 0 : s.qc_begin[h]);
     hp.kc_base = s.kc_begin[h];
     hp.n_items = items_of(d.N);
     hp.item_begin = item;
@@ -438,6 +442,8 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   p.out = out;
   p.segs = segs;
   p.seg_counts = cnts;
+  p.qmap = cache_i;
+  p.T = d.T;
   p.err = dev.err;
   p.ok_flag = ok_flag;
   p.wait_budget = kWaitBudget;
@@ -538,6 +544,7 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   }
   sp.corr_kmax = cl.corr_kmax;
   sp.corr_off = cl.corr_off;
+  sp.order_off = cl.order_off;
   CacheHeader& hd = sp.header;
   std::memset(&hd, 0, sizeof(hd));
   hd.magic = kCacheMagic;
@@ -547,6 +554,7 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   hd.T = d.T;
   hd.corr_kmax = cl.corr_kmax;
   hd.corr_off = cl.corr_off;
+  hd.order_off = cl.order_off;
   for (int h = 0; h < kMaxHeads; ++h) hd.probe_off[h] = h < d.H ? cl.probe_off[h] : -1;
   int launches = 0;
   cudaError_t e = launch_select(sp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), dino,

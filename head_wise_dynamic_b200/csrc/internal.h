@@ -38,6 +38,7 @@ struct CacheHeader {
   int32_t N, T;
   int32_t corr_kmax;        // width of the ranked tile list (0 = none)
   int32_t corr_off;         // int32 offset of the ranked tile list
+  int32_t order_off;        // int32 offset of the query-tile grouping order [T] (correspondence heads)
   int32_t probe_off[kMaxHeads];  // int32 offset of each probe head's key list (-1 = not a probe head)
 };
 static_assert(sizeof(CacheHeader) <= 512, "cache header too large");
@@ -60,8 +61,9 @@ constexpr uint32_t kSegCellMask = 0x10u;
 struct HeadPlan {
   int32_t head;       // head index h in [0, H)
   int32_t kind;       // saf3r_head_type
-  int32_t q_src;      // 0: caller Q rows are tokens; 1: derived cell-major Q rows (position heads)
-  int32_t q_base;     // derived Q row base (q_src == 1)
+  int32_t q_src;      // 0: caller Q rows are tokens; 1: derived cell-major Q rows (position heads);
+                      // 2: caller Q, each 64-row quarter of an item is the query tile qmap[4*item + quarter]
+  int32_t q_base;     // derived Q row base (q_src == 1); qmap offset (q_src == 2)
   int32_t kc_base;    // derived K/V row base
   int32_t n_items;    // work items (256 query rows each)
   int32_t item_begin; // first global item index
@@ -81,6 +83,8 @@ struct AttnParams {
   void* out;
   const Seg* segs;
   const int32_t* seg_counts;
+  const int32_t* qmap;    // query-tile order of the correspondence heads (in the cache)
+  int32_t T;              // 64-token tiles
   int* err;
   const int* ok_flag;  // nonzero: cache check passed (NULL: no check)
   long long wait_budget;
@@ -97,6 +101,7 @@ struct SelectPlan {
   int probe_off[kMaxHeads];
   int corr_kmax;
   int corr_off;
+  int order_off;
   CacheHeader header;
 };
 
@@ -142,8 +147,8 @@ cudaError_t launch_derived(const DerivedArgs& a, bool any_scan, const uint16_t* 
                            uint16_t* qc, int* err, int num_sms, cudaStream_t stream, int* n_launch);
 cudaError_t launch_plan_position(int n_items, int S, int gh, int gw, int ns, int N, int R, int cap, Seg* segs,
                                  int* counts, cudaStream_t stream);
-cudaError_t launch_plan_corr(const int32_t* ranked, int kmax, int kt, int T, int N, int V, int ns, int S,
-                             Seg* segs, int cap, int* counts, int* err, cudaStream_t stream);
+cudaError_t launch_plan_corr(const int32_t* ranked, const int32_t* order, int kmax, int kt, int T, int N, int V,
+                             int ns, int S, Seg* segs, int cap, int* counts, int* err, cudaStream_t stream);
 size_t nmse_workspace_bytes(int H);
 cudaError_t launch_nmse(const float* full, const float* sparse, int H, long long per_head, double* part,
                         double* out, cudaStream_t stream);

@@ -188,10 +188,11 @@ __global__ void plan_position_kernel(int n_items, int S, int gh, int gw, int ns,
   counts[m] = n;
 }
 
-// Key runs of every 256-row item of a correspondence head: the union of the four
+// Key runs of every 256-row item of a correspondence head: the union of its four
 // query tiles' selected key tiles (ascending, with the quarters that keep each),
-// then the special tokens.
-__global__ void __launch_bounds__(256) plan_corr_kernel(const int32_t* __restrict__ ranked, int kmax, int kt, int T,
+// then the special tokens.  Quarter q of item m is query tile order[4m + q].
+__global__ void __launch_bounds__(256) plan_corr_kernel(const int32_t* __restrict__ ranked,
+                                                        const int32_t* __restrict__ order, int kmax, int kt, int T,
                                                         int N, int V, int ns, int S, Seg* __restrict__ segs,
                                                         int cap, int* __restrict__ counts, int* err) {
   extern __shared__ uint32_t memb[];  // [T]
@@ -201,8 +202,12 @@ __global__ void __launch_bounds__(256) plan_corr_kernel(const int32_t* __restric
   __syncthreads();
   for (int e = threadIdx.x; e < 4 * kt; e += blockDim.x) {
     const int q = e / kt, r = e - q * kt;
-    const int u = 4 * m + q;
-    if (u >= T) continue;
+    if (4 * m + q >= T) continue;
+    const int u = order[4 * m + q];
+    if (u < 0 || u >= T) {
+      atomicCAS(err, 0, SAF3R_ERR_INDEX);
+      continue;
+    }
     const int v = ranked[static_cast<size_t>(u) * kmax + r];
     if (v < 0 || v >= T) {
       atomicCAS(err, 0, SAF3R_ERR_INDEX);
@@ -328,8 +333,8 @@ cudaError_t launch_plan_position(int n_items, int S, int gh, int gw, int ns, int
   return cudaGetLastError();
 }
 
-cudaError_t launch_plan_corr(const int32_t* ranked, int kmax, int kt, int T, int N, int V, int ns, int S,
-                             Seg* segs, int cap, int* counts, int* err, cudaStream_t stream) {
+cudaError_t launch_plan_corr(const int32_t* ranked, const int32_t* order, int kmax, int kt, int T, int N, int V,
+                             int ns, int S, Seg* segs, int cap, int* counts, int* err, cudaStream_t stream) {
   const int n_items = (T + 3) / 4;
   const size_t smem = sizeof(uint32_t) * T;
   if (smem > 48 * 1024) {
@@ -337,7 +342,8 @@ cudaError_t launch_plan_corr(const int32_t* ranked, int kmax, int kt, int T, int
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  plan_corr_kernel<<<n_items, 256, smem, stream>>>(ranked, kmax, kt, T, N, V, ns, S, segs, cap, counts, err);
+  plan_corr_kernel<<<n_items, 256, smem, stream>>>(ranked, order, kmax, kt, T, N, V, ns, S, segs, cap, counts,
+                                                   err);
   return cudaGetLastError();
 }
 

@@ -329,6 +329,124 @@ __global__ void __launch_bounds__(256) tile_topk_kernel(const float* __restrict_
   }
 }
 
+// ---- query-tile grouping of the correspondence heads (a scheduling aid, cached with the indices)
+//
+// Four query tiles share one 256-row attention work item and the union of their key
+// tiles.  Tiles whose ranked lists overlap are put together: sort by a canonical key
+// (the smallest tile index among the first `r` ranks), then, inside windows of 64
+// consecutive tiles, greedily grow groups of four by shared-tile counts.  The order
+// changes only which rows share an item, never a result.
+constexpr int kGroupWindow = 64;
+constexpr int kMaxSortTiles = 16384;
+
+__global__ void __launch_bounds__(1024) corr_sort_kernel(const int32_t* __restrict__ ranked, int T, int kmax,
+                                                         int r, int32_t* __restrict__ order) {
+  extern __shared__ unsigned long long keys[];  // [pow2 >= T]
+  int n2 = 1;
+  while (n2 < T) n2 <<= 1;
+  for (int u = threadIdx.x; u < n2; u += blockDim.x) {
+    unsigned long long k = ~0ull;
+    if (u < T) {
+      int mn = 0x7fffffff;
+      for (int i = 0; i < r; ++i) mn = min(mn, ranked[static_cast<size_t>(u) * kmax + i]);
+      k = (static_cast<unsigned long long>(static_cast<uint32_t>(mn)) << 32) | static_cast<uint32_t>(u);
+    }
+    keys[u] = k;
+  }
+  __syncthreads();
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const unsigned long long a = keys[i], b = keys[j];
+          if ((a > b) == up) {
+            keys[i] = b;
+            keys[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int u = threadIdx.x; u < T; u += blockDim.x) order[u] = static_cast<int32_t>(keys[u] & 0xffffffffu);
+}
+
+__global__ void corr_bitset_kernel(const int32_t* __restrict__ ranked, int T, int kmax, int words,
+                                   uint32_t* __restrict__ bits) {
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < static_cast<long long>(T) * kmax;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int u = static_cast<int>(e / kmax);
+    const int v = ranked[e];
+    if (v >= 0 && v < T) atomicOr(&bits[static_cast<size_t>(u) * words + (v >> 5)], 1u << (v & 31));
+  }
+}
+
+__global__ void __launch_bounds__(256) corr_group_kernel(const uint32_t* __restrict__ bits, int T, int words,
+                                                         const int32_t* __restrict__ sorted,
+                                                         int32_t* __restrict__ order) {
+  __shared__ uint16_t inter[kGroupWindow][kGroupWindow];
+  __shared__ int tiles[kGroupWindow];
+  const int w0 = blockIdx.x * kGroupWindow;
+  const int n = min(kGroupWindow, T - w0);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) tiles[i] = sorted[w0 + i];
+  __syncthreads();
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int a = e / n, b = e - a * n;
+    if (b < a) continue;
+    const uint32_t* ba = bits + static_cast<size_t>(tiles[a]) * words;
+    const uint32_t* bb = bits + static_cast<size_t>(tiles[b]) * words;
+    int c = 0;
+    for (int w = 0; w < words; ++w) c += __popc(ba[w] & bb[w]);
+    inter[a][b] = inter[b][a] = static_cast<uint16_t>(min(c, 65535));
+  }
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  // one warp: greedy groups of four inside the window; lane l owns candidates l and l + 32
+  const int lane = threadIdx.x;
+  bool left0 = lane < n, left1 = lane + 32 < n;
+  int out = w0;
+  for (int u = 0; u < n; ++u) {
+    const bool u_left = __shfl_sync(0xffffffffu, (u & 31) < 32 ? ((u < 32) ? left0 : left1) : false, u & 31);
+    if (!u_left) continue;
+    if (lane == (u & 31)) {
+      if (u < 32) left0 = false; else left1 = false;
+    }
+    if (lane == 0) order[out] = tiles[u];
+    ++out;
+    int sc0 = left0 ? inter[u][lane] : -1;
+    int sc1 = left1 ? inter[u][lane + 32] : -1;
+    for (int k = 0; k < 3; ++k) {
+      // argmax over the window (ties to the earlier position)
+      int best = sc0 >= sc1 ? sc0 : sc1;
+      int pos = sc0 >= sc1 ? lane : lane + 32;
+      if (best < 0) pos = 1 << 20;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const int ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int op = __shfl_xor_sync(0xffffffffu, pos, o);
+        if (ob > best || (ob == best && op < pos)) {
+          best = ob;
+          pos = op;
+        }
+      }
+      if (best < 0) break;
+      if (lane == 0) order[out] = tiles[pos];
+      ++out;
+      if (pos == lane) left0 = false;
+      if (pos == lane + 32) left1 = false;
+      sc0 = left0 ? sc0 + inter[pos][lane] : -1;
+      sc1 = left1 ? sc1 + inter[pos][lane + 32] : -1;
+    }
+  }
+}
+
+__global__ void identity_order_kernel(int T, int32_t* order) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u < T) order[u] = u;
+}
+
 __global__ void cache_header_kernel(CacheHeader h, CacheHeader* dst) {
   if (threadIdx.x == 0) *dst = h;
 }
@@ -342,7 +460,13 @@ size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr) {
   b = (b + 255) & ~size_t(255);
   b += static_cast<size_t>(n_probe) * N * sizeof(float);
   b = (b + 255) & ~size_t(255);
-  if (corr) b += static_cast<size_t>(T) * dim * sizeof(float);
+  if (corr) {
+    b += static_cast<size_t>(T) * dim * sizeof(float);
+    b = (b + 255) & ~size_t(255);
+    b += static_cast<size_t>(T) * ((T + 31) / 32) * sizeof(uint32_t);  // grouping bitsets
+    b = (b + 255) & ~size_t(255);
+    b += static_cast<size_t>(T) * sizeof(int32_t);                      // sorted tiles
+  }
   return b + 256;
 }
 
@@ -399,6 +523,34 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
     tile_topk_kernel<<<(sp.T + R - 1) / R, 256, smem, stream>>>(tilevec, sp.T, sp.dim, R, sp.corr_kmax,
                                                                 cache + sp.corr_off);
     *n_launch += 2;
+    // query-tile grouping for the attention work items
+    size_t goff = static_cast<size_t>(reinterpret_cast<uint8_t*>(tilevec) - ws) +
+                  static_cast<size_t>(sp.T) * sp.dim * sizeof(float);
+    goff = (goff + 255) & ~size_t(255);
+    const int words = (sp.T + 31) / 32;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(ws + goff);
+    goff += static_cast<size_t>(sp.T) * words * sizeof(uint32_t);
+    goff = (goff + 255) & ~size_t(255);
+    int32_t* sorted = reinterpret_cast<int32_t*>(ws + goff);
+    int32_t* order = cache + sp.order_off;
+    if (sp.T <= kMaxSortTiles) {
+      int n2 = 1;
+      while (n2 < sp.T) n2 <<= 1;
+      const size_t ssmem = sizeof(unsigned long long) * n2;
+      e = cudaFuncSetAttribute(corr_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssmem));
+      if (e != cudaSuccess) return e;
+      corr_sort_kernel<<<1, 1024, ssmem, stream>>>(cache + sp.corr_off, sp.T, sp.corr_kmax,
+                                                   sp.corr_kmax > 1 ? sp.corr_kmax / 2 : 1, sorted);
+      e = cudaMemsetAsync(bits, 0, static_cast<size_t>(sp.T) * words * sizeof(uint32_t), stream);
+      if (e != cudaSuccess) return e;
+      corr_bitset_kernel<<<148, 256, 0, stream>>>(cache + sp.corr_off, sp.T, sp.corr_kmax, words, bits);
+      corr_group_kernel<<<(sp.T + kGroupWindow - 1) / kGroupWindow, 256, 0, stream>>>(bits, sp.T, words, sorted,
+                                                                                      order);
+      *n_launch += 3;
+    } else {
+      identity_order_kernel<<<(sp.T + 255) / 256, 256, 0, stream>>>(sp.T, order);
+      *n_launch += 1;
+    }
   }
   return cudaGetLastError();
 }
