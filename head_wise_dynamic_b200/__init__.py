@@ -172,6 +172,17 @@ def saf3r_select_kv(layout, cfg, q, k, dino, cache, workspace, stream=None):
     _check(st, "saf3r_select_kv")
 
 
+def saf3r_select_kv_static(layout, cfg, q, k, dino, cache, stream=None):
+    """saf3r_select_kv for callers that cannot allocate a device workspace: the scratch
+    comes from a fixed 16 MiB array inside the library (see include/saf3r.h for the limit,
+    the first-call set-up and the rule that overlapping calls race)."""
+    f = lib().saf3r_select_kv_static
+    f.argtypes = [ctypes.POINTER(saf3r_layout), ctypes.POINTER(saf3r_head_cfg)] + [ctypes.c_void_p] * 5
+    f.restype = ctypes.c_int
+    st = f(ctypes.byref(layout_of(layout)), _cfg(cfg), _ptr(q), _ptr(k), _ptr(dino), _ptr(cache), _stream(stream))
+    _check(st, "saf3r_select_kv_static")
+
+
 def saf3r_sparse_attn(layout, cfg, cache, q, k, v, out, workspace, stream=None, out_is_fp32: Optional[bool] = None):
     if out_is_fp32 is None:
         import torch
