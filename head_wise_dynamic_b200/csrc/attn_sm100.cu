@@ -332,69 +332,56 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint
 }
 
 // ------------------------------------------------------------------ softmax (one thread per row)
-__device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, uint32_t tmem, int warp, int lane) {
+//
+// Key masks, by head kind (the loop is instantiated once per kind, so a head pays only
+// for the masks it can have):
+//   kMaskPlain     - only the ragged end of a run (probe, stride and dense heads)
+//   kMaskTiles     - + tiles this row's quarter does not keep, special tokens already
+//                    counted inside a tile (correspondence heads)
+//   kMaskCells     - + neighbour cells of this row's grid cell (position heads)
+constexpr int kMaskPlain = 0, kMaskTiles = 1, kMaskCells = 2;
+
+struct RowCtx {
+  int t, lane, quarter;
+  uint32_t tS, tP, tO;
+  int nb_lo[2 * kMaxRadius + 1], nb_hi[2 * kMaxRadius + 1];  // kMaskCells: kept derived rows [lo, hi)
+};
+
+template <int kMask>
+__device__ __forceinline__ uint64_t key_mask(const Half& hb, const RowCtx& rc) {
+  if (!hb.have) return 0ull;
+  if (kMask == kMaskTiles && !((hb.s.flags >> rc.quarter) & 1u)) return 0ull;
+  uint64_t v = hb.cnt >= 64 ? ~0ull : ((1ull << hb.cnt) - 1ull);
+  if (kMask == kMaskTiles) {
+    const int lo = (hb.s.flags >> 8) & 0xFF, hi = (hb.s.flags >> 16) & 0xFF;
+    if (hi > lo) v &= ~range_bits(max(lo - hb.off, 0), min(hi - hb.off, 64));
+  }
+  if (kMask == kMaskCells && (hb.s.flags & kSegCellMask)) {
+    const int base = hb.s.row0 + hb.off;
+    uint64_t nb = 0ull;
+#pragma unroll
+    for (int x = 0; x < 2 * kMaxRadius + 1; ++x)
+      nb |= range_bits(max(rc.nb_lo[x] - base, 0), min(rc.nb_hi[x] - base, hb.cnt));
+    v &= nb;
+  }
+  return v;
+}
+
+// All key blocks of one item for one row; returns false if a wait gave up.
+template <int kMask>
+__device__ __forceinline__ bool softmax_blocks(const AttnParams& p, AttnSmem& sm, ItemInfo& it, const RowCtx& rc,
+                                               uint32_t& sfull_c, uint32_t& odone_c, float& l_out) {
   volatile int* abort = &sm.abort;
   const long long budget = p.wait_budget;
-  const int t = (warp - 4) >> 2;
-  const int wq = warp & 3;
-  const int r = wq * 32 + lane;            // row inside the 128-row tile
-  const int quarter = (t * 128 + r) >> 6;  // 64-row quarter of the 256-row item
-  const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-  const uint32_t tS = tmem + lane_off + t * 256;
-  const uint32_t tP = tS + 128;
-  const uint32_t tO = tS + 192;
-  uint32_t sfull_c = 0, odone_c = 0;
+  const int t = rc.t, lane = rc.lane;
+  const uint32_t tS = rc.tS, tP = rc.tP, tO = rc.tO;
   bool ok = true;
-
-  for (int item = blockIdx.x; ok && item < p.total_items; item += gridDim.x) {
-    ItemInfo it = item_info(p, item);
-    const HeadPlan& hp = p.heads[it.hi];
-    const int qrow = it.q0 + t * 128 + r;
-
-    // per-row neighbourhood intervals (position heads): kept derived rows [lo, hi)
-    int nb_lo[2 * kMaxRadius + 1], nb_hi[2 * kMaxRadius + 1];
-    {
-      const bool patch_row = hp.kind == SAF3R_POSITION && qrow < p.P * p.S && p.S > 1;
-      const int cell = patch_row ? qrow / p.S : 0;
-      const int qr = cell / p.gw, qc = cell - qr * p.gw;
-      const int R = hp.radius;
-#pragma unroll
-      for (int x = 0; x < 2 * kMaxRadius + 1; ++x) {
-        const int dr = x - kMaxRadius;
-        const int rr = qr + dr;
-        const bool use = patch_row && dr >= -R && dr <= R && rr >= 0 && rr < p.gh;
-        const int ca = rr * p.gw + max(qc - R, 0);
-        const int cb = rr * p.gw + min(qc + R, p.gw - 1);
-        nb_lo[x] = use ? hp.nb_base + ca * (p.S - 1) : 0;
-        nb_hi[x] = use ? hp.nb_base + (cb + 1) * (p.S - 1) : 0;
-      }
-    }
-
-    float m = -INFINITY;  // running max, log2 units
-    float l = 0.f;        // running row sum
-    for (int j = 0; j < it.nblk; ++j) {
-      // kept-key masks of the two halves of this block
-      uint64_t valid[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const Half hb = it.w.next();
-        valid[h] = 0ull;
-        if (hb.have && ((hb.s.flags >> quarter) & 1u)) {
-          uint64_t v = range_bits(0, hb.cnt);
-          const int lo = (hb.s.flags >> 8) & 0xFF, hi = (hb.s.flags >> 16) & 0xFF;
-          if (hi > lo) v &= ~range_bits(max(lo - hb.off, 0), min(hi - hb.off, 64));
-          if (hb.s.flags & kSegCellMask) {
-            const int base = hb.s.row0 + hb.off;
-            uint64_t nb = 0ull;
-#pragma unroll
-            for (int x = 0; x < 2 * kMaxRadius + 1; ++x)
-              nb |= range_bits(max(nb_lo[x] - base, 0), min(nb_hi[x] - base, hb.cnt));
-            v &= nb;
-          }
-          valid[h] = v;
-        }
-      }
-
+  float m = -INFINITY;  // running max, log2 units
+  float l = 0.f;        // running row sum
+  for (int j = 0; j < it.nblk; ++j) {
+    uint64_t valid[2];
+    valid[0] = key_mask<kMask>(it.w.next(), rc);
+    valid[1] = key_mask<kMask>(it.w.next(), rc);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], sfull_c & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
         ok = false;
         break;
@@ -403,14 +390,14 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
       tc_fence_after();
       float s[128];
       {
-        uint32_t raw[32];
+        uint32_t raw[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tS + c * 32, raw);
-          tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, raw[c]);
+        tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[i]);
-        }
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[c][i]);
       }
       tc_fence_before();
       __syncwarp();
@@ -441,15 +428,19 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
         rescale = true;
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
+      // 8 independent partial row sums: a single running sum would be a chain of 128 dependent adds
       uint32_t pk[64];
-      float rs = 0.f;
+      float rp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rp[i] = 0.f;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         const float e0 = fast_exp2(fmaf(s[2 * i], kScaleLog2, -m_use));
         const float e1 = fast_exp2(fmaf(s[2 * i + 1], kScaleLog2, -m_use));
-        rs += e0 + e1;
+        rp[i & 7] += e0 + e1;
         pk[i] = pack_bf16x2(e0, e1);
       }
+      const float rs = ((rp[0] + rp[1]) + (rp[2] + rp[3])) + ((rp[4] + rp[5]) + (rp[6] + rp[7]));
       l = l * alpha + rs;
 
       if (j > 0) {
@@ -484,6 +475,56 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[t]);
+  }
+  l_out = l;
+  return ok;
+}
+
+__device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, uint32_t tmem, int warp, int lane) {
+  volatile int* abort = &sm.abort;
+  const long long budget = p.wait_budget;
+  RowCtx rc;
+  rc.t = (warp - 4) >> 2;
+  rc.lane = lane;
+  const int t = rc.t;
+  const int wq = warp & 3;
+  const int r = wq * 32 + lane;   // row inside the 128-row tile
+  rc.quarter = (t * 128 + r) >> 6;  // 64-row quarter of the 256-row item
+  const int quarter = rc.quarter;
+  const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+  rc.tS = tmem + lane_off + t * 256;
+  rc.tP = rc.tS + 128;
+  rc.tO = rc.tS + 192;
+  const uint32_t tO = rc.tO;
+  uint32_t sfull_c = 0, odone_c = 0;
+  bool ok = true;
+
+  for (int item = blockIdx.x; ok && item < p.total_items; item += gridDim.x) {
+    ItemInfo it = item_info(p, item);
+    const HeadPlan& hp = p.heads[it.hi];
+    const int qrow = it.q0 + t * 128 + r;
+    float l = 0.f;
+    if (hp.kind == SAF3R_POSITION) {
+      // neighbour cells of this row's grid cell, as kept derived rows [lo, hi)
+      const bool patch_row = qrow < p.P * p.S && p.S > 1;
+      const int cell = patch_row ? qrow / p.S : 0;
+      const int qr = cell / p.gw, qc = cell - qr * p.gw;
+      const int R = hp.radius;
+#pragma unroll
+      for (int x = 0; x < 2 * kMaxRadius + 1; ++x) {
+        const int dr = x - kMaxRadius;
+        const int rr = qr + dr;
+        const bool use = patch_row && dr >= -R && dr <= R && rr >= 0 && rr < p.gh;
+        const int ca = rr * p.gw + max(qc - R, 0);
+        const int cb = rr * p.gw + min(qc + R, p.gw - 1);
+        rc.nb_lo[x] = use ? hp.nb_base + ca * (p.S - 1) : 0;
+        rc.nb_hi[x] = use ? hp.nb_base + (cb + 1) * (p.S - 1) : 0;
+      }
+      ok = softmax_blocks<kMaskCells>(p, sm, it, rc, sfull_c, odone_c, l);
+    } else if (hp.kind == SAF3R_CORR) {
+      ok = softmax_blocks<kMaskTiles>(p, sm, it, rc, sfull_c, odone_c, l);
+    } else {
+      ok = softmax_blocks<kMaskPlain>(p, sm, it, rc, sfull_c, odone_c, l);
     }
     if (!ok) break;
 
