@@ -16,14 +16,16 @@
 //
 // Warp roles (12 warps, three warpgroups):
 //   warp 0      TMA producer: Q tiles, then K and V blocks into a 4-stage ring
-//   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
+//   warp 1      MMA issuer (one thread): O_t += P_t V, then S_t = Q_t K^T of the next block
 //   warps 2-3   idle (their registers go to the softmax warpgroups)
-//   warps 4-7   softmax of tile 0 (one thread per row; warp w reads TMEM lanes 32*(w%4)..+31)
-//   warps 8-11  softmax of tile 1
-// TMEM (512 columns): per tile t, S_t (128 fp32 cols), P_t (64 cols of packed
-// bf16 pairs), O_t (64 fp32 cols).  The two softmax groups alternate with the
-// tensor core: while group 0 turns S_0 into P_0, the tensor core runs group
-// 1's products, and the other way round.
+//   warps 4-11  softmax: warp w owns rows 32*(w%4)..+31 of a tile (the TMEM lanes it may
+//               read) and key half (w-4)/4 of every 128-key block; all eight warps work
+//               on tile 0, then on tile 1, so each tile's products run on the tensor
+//               core while the other tile's exponentials run on the SFUs.
+// TMEM (512 columns): per tile t, S_t (128 fp32 cols; each warp writes its bf16 P over the
+// first 32 columns of its own key half once it has read them) and two accumulators
+// O_t,a / O_t,b (64 fp32 cols each), one per key half, merged with the halves' running
+// maxima and sums when the item ends.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -49,7 +51,9 @@ struct AttnSmem {
   uint8_t v[kStages][kTileBytes];
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t pair[4];           // the two warps sharing rows 32*w..+31 (w = warp % 4) meet here at an item's end
+  float stats[2][2][128][2];  // [key half][tile][row] = (running max, running sum) for the final merge
   uint32_t tmem_base;
   int abort;
 };
@@ -222,16 +226,14 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm,
 
 // ------------------------------------------------------------------ MMA issuer (one thread)
 //
-// For each key block and each tile in turn: O_t += P_t V once softmax t has written P_t,
-// then S_t = Q_t K^T of the next block.  The two softmax groups so alternate with the
-// tensor core: while group t computes, the tensor core runs the other tile's products.
-// This thread sits on that critical path, so it does nothing but wait, add descriptor
-// offsets and issue: every product covers the whole 128-key block (keys a row does not
-// keep are masked in its softmax and get P = 0).
+// For each key block and each tile in turn: O_t,a += P_t,a V[0:64] and O_t,b += P_t,b V[64:128]
+// once all eight softmax warps have written P_t, then S_t = Q_t K^T of the next block (it
+// overwrites P_t, which the products just issued have read: this thread's products execute
+// in issue order).  This thread sits on the critical path, so it does nothing but wait, add
+// descriptor offsets and issue; every product covers the whole block (keys a row does not
+// keep get P = 0).
 struct MmaState {
-  uint32_t sfree_c[2] = {0, 0};
   uint32_t pfull_c[2] = {0, 0};
-  uint32_t qk_done[2] = {0, 0};
 };
 
 // Shared-memory descriptors of the operand tiles, computed once: a K-step of 16 keys or 16
@@ -243,23 +245,13 @@ struct Descs {
 };
 constexpr uint64_t kStageDesc = kTileBytes >> 4;
 
-// S_t = Q_t K^T for one 128-key block; commits s_full[t].
-__device__ __forceinline__ bool issue_qk(const AttnParams& p, AttnSmem& sm, MmaState& st, const Descs& d,
-                                         uint32_t tmem, int t, uint32_t stage) {
-  if (st.qk_done[t] > 0) {
-    if (!mbar_wait(&sm.s_free[t], st.sfree_c[t] & 1, &sm.abort, p.err, p.wait_budget, SAF3R_ERR_TIMEOUT))
-      return false;
-    ++st.sfree_c[t];
-    tc_fence_after();
-  }
+// S_t = Q_t K^T for one 128-key block.
+__device__ __forceinline__ void issue_qk(const Descs& d, uint32_t tmem, int t, uint32_t stage) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
   const uint64_t dq = d.q[t];
   const uint64_t dk = d.k0 + stage * kStageDesc;
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + t * 256, dq + 2 * kk, dk + 2 * kk, idesc, kk > 0 ? 1u : 0u);
-  mma_commit(&sm.s_full[t]);
-  ++st.qk_done[t];
-  return true;
 }
 
 __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint32_t tmem) {
@@ -282,7 +274,10 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint
       const uint32_t stage = kv_c % kStages, ph = (kv_c / kStages) & 1;
       if (!mbar_wait(&sm.k_full[stage], ph, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) break;
       tc_fence_after();
-      if (!issue_qk(p, sm, st, d, tmem, 0, stage) || !issue_qk(p, sm, st, d, tmem, 1, stage)) break;
+      issue_qk(d, tmem, 0, stage);
+      mma_commit(&sm.s_full[0]);
+      issue_qk(d, tmem, 1, stage);
+      mma_commit(&sm.s_full[1]);
       mma_commit(&sm.k_empty[stage]);
       if (nblk == 1) mma_commit(&sm.q_empty);
     }
@@ -309,14 +304,19 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint
         }
         ++st.pfull_c[t];
         tc_fence_after();
-        const uint32_t o_col = tmem + t * 256 + 192, p_col = tmem + t * 256 + 128;
-        mma_ts(o_col, p_col, dv, idesc_pv, j > 0 ? 1u : 0u);
+        const uint32_t s_col = tmem + t * 256, o_col = s_col + 128;
+        // key half a: P in S columns 0..31, keys 0..63 of V; key half b: S columns 64..95, keys 64..127
+        mma_ts(o_col, s_col, dv, idesc_pv, j > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < 8; ++kk) mma_ts(o_col, p_col + kk * 8, dv + 128 * kk, idesc_pv, 1u);
-        mma_commit(&sm.o_done[t]);
-        if (has_next && !issue_qk(p, sm, st, d, tmem, t, ns)) {
-          ok = false;
-          break;
+        for (int kk = 1; kk < 4; ++kk) mma_ts(o_col, s_col + kk * 8, dv + 128 * kk, idesc_pv, 1u);
+        mma_ts(o_col + 64, s_col + 64, dv + 128 * 4, idesc_pv, j > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 1; kk < 4; ++kk) mma_ts(o_col + 64, s_col + 64 + kk * 8, dv + 128 * (4 + kk), idesc_pv, 1u);
+        if (has_next) {
+          issue_qk(d, tmem, t, ns);
+          mma_commit(&sm.s_full[t]);
+        } else {
+          mma_commit(&sm.o_done[t]);
         }
       }
       if (!ok) break;
@@ -331,7 +331,7 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint
   }
 }
 
-// ------------------------------------------------------------------ softmax (one thread per row)
+// ------------------------------------------------------------------ softmax (one thread per row and key half)
 //
 // Key masks, by head kind (the loop is instantiated once per kind, so a head pays only
 // for the masks it can have):
@@ -340,17 +340,21 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint
 //                    counted inside a tile (correspondence heads)
 //   kMaskCells     - + neighbour cells of this row's grid cell (position heads)
 constexpr int kMaskPlain = 0, kMaskTiles = 1, kMaskCells = 2;
+constexpr int kNbIntervals = 2 * kMaxRadius + 1;
 
 struct RowCtx {
-  int t, lane, quarter;
-  uint32_t tS, tP, tO;
-  int nb_lo[2 * kMaxRadius + 1], nb_hi[2 * kMaxRadius + 1];  // kMaskCells: kept derived rows [lo, hi)
+  int kh;            // key half of every block this warp owns (0: keys 0..63, 1: keys 64..127)
+  int r;             // row inside each 128-row tile
+  int lane;
+  uint32_t lane_off; // TMEM lane field of this warp
+  int nb_lo[2][kNbIntervals], nb_hi[2][kNbIntervals];  // position heads: kept derived rows [lo, hi) per tile
 };
 
 template <int kMask>
-__device__ __forceinline__ uint64_t key_mask(const Half& hb, const RowCtx& rc) {
+__device__ __forceinline__ uint64_t key_mask(const Half& hb, const RowCtx& rc, int t) {
   if (!hb.have) return 0ull;
-  if (kMask == kMaskTiles && !((hb.s.flags >> rc.quarter) & 1u)) return 0ull;
+  const int quarter = (t * 128 + rc.r) >> 6;
+  if (kMask == kMaskTiles && !((hb.s.flags >> quarter) & 1u)) return 0ull;
   uint64_t v = hb.cnt >= 64 ? ~0ull : ((1ull << hb.cnt) - 1ull);
   if (kMask == kMaskTiles) {
     const int lo = (hb.s.flags >> 8) & 0xFF, hi = (hb.s.flags >> 16) & 0xFF;
@@ -360,186 +364,210 @@ __device__ __forceinline__ uint64_t key_mask(const Half& hb, const RowCtx& rc) {
     const int base = hb.s.row0 + hb.off;
     uint64_t nb = 0ull;
 #pragma unroll
-    for (int x = 0; x < 2 * kMaxRadius + 1; ++x)
-      nb |= range_bits(max(rc.nb_lo[x] - base, 0), min(rc.nb_hi[x] - base, hb.cnt));
+    for (int x = 0; x < kNbIntervals; ++x)
+      nb |= range_bits(max(rc.nb_lo[t][x] - base, 0), min(rc.nb_hi[t][x] - base, hb.cnt));
     v &= nb;
   }
   return v;
 }
 
-// All key blocks of one item for one row; returns false if a wait gave up.
+struct SoftmaxState {
+  uint32_t sfull_c[2] = {0, 0};
+  uint32_t odone_c = 0;
+  uint32_t pair_c = 0;
+};
+
+// One 64-key half-block of one tile for this thread's row: masks, running max, exponentials,
+// P (bf16) written over the half's first 32 S columns, arrival on p_full[t].
 template <int kMask>
-__device__ __forceinline__ bool softmax_blocks(const AttnParams& p, AttnSmem& sm, ItemInfo& it, const RowCtx& rc,
-                                               uint32_t& sfull_c, uint32_t& odone_c, float& l_out) {
-  volatile int* abort = &sm.abort;
-  const long long budget = p.wait_budget;
-  const int t = rc.t, lane = rc.lane;
-  const uint32_t tS = rc.tS, tP = rc.tP, tO = rc.tO;
-  bool ok = true;
-  float m = -INFINITY;  // running max, log2 units
-  float l = 0.f;        // running row sum
-  for (int j = 0; j < it.nblk; ++j) {
-    uint64_t valid[2];
-    valid[0] = key_mask<kMask>(it.w.next(), rc);
-    valid[1] = key_mask<kMask>(it.w.next(), rc);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], sfull_c & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
-        ok = false;
-        break;
-      }
-      ++sfull_c;
-      tc_fence_after();
-      float s[128];
-      {
-        uint32_t raw[4][32];
+__device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, SoftmaxState& ss, uint32_t tmem,
+                                             const RowCtx& rc, int t, int j, uint64_t valid, float& m, float& l) {
+  if (!__all_sync(0xffffffffu,
+                  mbar_wait(&sm.s_full[t], ss.sfull_c[t] & 1, &sm.abort, p.err, p.wait_budget, SAF3R_ERR_TIMEOUT)))
+    return false;
+  ++ss.sfull_c[t];
+  tc_fence_after();
+  const uint32_t tS = tmem + rc.lane_off + t * 256 + rc.kh * 64;
+  float s[64];
+  {
+    uint32_t raw[2][32];
+    tmem_ld32(tS, raw[0]);
+    tmem_ld32(tS + 32, raw[1]);
+    tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, raw[c]);
-        tmem_wait_ld();
+    for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[c][i]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[t]);
-
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (valid[h] != ~0ull) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (!((valid[h] >> i) & 1ull)) s[h * 64 + i] = -INFINITY;
-        }
-      }
-      float mp[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mp[i] = s[i];
-#pragma unroll
-      for (int i = 8; i < 128; ++i) mp[i & 7] = fmaxf(mp[i & 7], s[i]);
-      float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      mx *= kScaleLog2;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (j == 0) {
-        m = mx;
-      } else if (mx > m + kRescaleThreshold) {
-        alpha = fast_exp2(m - mx);
-        m = mx;
-        rescale = true;
-      }
-      const float m_use = (m == -INFINITY) ? 0.f : m;
-      // 8 independent partial row sums: a single running sum would be a chain of 128 dependent adds
-      uint32_t pk[64];
-      float rp[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) rp[i] = 0.f;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float e0 = fast_exp2(fmaf(s[2 * i], kScaleLog2, -m_use));
-        const float e1 = fast_exp2(fmaf(s[2 * i + 1], kScaleLog2, -m_use));
-        rp[i & 7] += e0 + e1;
-        pk[i] = pack_bf16x2(e0, e1);
-      }
-      const float rs = ((rp[0] + rp[1]) + (rp[2] + rp[3])) + ((rp[4] + rp[5]) + (rp[6] + rp[7]));
-      l = l * alpha + rs;
-
-      if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], odone_c & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
-          ok = false;
-          break;
-        }
-        ++odone_c;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
-          uint32_t o[32];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tO + c * 32, o);
-          }
-        }
-      }
-      {
-        uint32_t half[32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) half[i] = pk[c * 32 + i];
-          tmem_st32(tP + c * 32, half);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[t]);
+      for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[c][i]);
   }
-  l_out = l;
-  return ok;
+  if (valid != ~0ull) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      if (!((valid >> i) & 1ull)) s[i] = -INFINITY;
+  }
+  float mp[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mp[i] = s[i];
+#pragma unroll
+  for (int i = 8; i < 64; ++i) mp[i & 7] = fmaxf(mp[i & 7], s[i]);
+  const float mx =
+      fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
+      kScaleLog2;
+  float alpha = 1.f;
+  bool rescale = false;
+  if (j == 0) {
+    m = mx;
+  } else if (mx > m + kRescaleThreshold) {
+    alpha = fast_exp2(m - mx);  // m may be -inf: alpha = 0
+    m = mx;
+    rescale = true;
+  }
+  if (__any_sync(0xffffffffu, rescale)) {
+    // rare: the running max grew by more than the threshold.  O_t of this half already holds the
+    // previous blocks' products (s_full of this block was committed after them); rescale it.
+    const uint32_t tO = tmem + rc.lane_off + t * 256 + 128 + rc.kh * 64;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      uint32_t o[16];
+      tmem_ld16(tO + q * 16, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+      tmem_st16(tO + q * 16, o);
+    }
+  }
+  const float m_use = (m == -INFINITY) ? 0.f : m;
+  // 8 independent partial row sums: a single running sum would be a chain of dependent adds
+  uint32_t pk[32];
+  float rp[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) rp[i] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float e0 = fast_exp2(fmaf(s[2 * i], kScaleLog2, -m_use));
+    const float e1 = fast_exp2(fmaf(s[2 * i + 1], kScaleLog2, -m_use));
+    rp[i & 7] += e0 + e1;
+    pk[i] = pack_bf16x2(e0, e1);
+  }
+  l = l * alpha + (((rp[0] + rp[1]) + (rp[2] + rp[3])) + ((rp[4] + rp[5]) + (rp[6] + rp[7])));
+  tmem_st32(tS, pk);
+  tmem_wait_st();
+  tc_fence_before();
+  __syncwarp();
+  if (rc.lane == 0) mbar_arrive(&sm.p_full[t]);
+  return true;
+}
+
+// All key blocks of one item: tile 0 then tile 1 for every block.
+template <int kMask>
+__device__ __forceinline__ bool softmax_blocks(const AttnParams& p, AttnSmem& sm, SoftmaxState& ss, uint32_t tmem,
+                                               ItemInfo& it, const RowCtx& rc, float (&m)[2], float (&l)[2]) {
+  for (int j = 0; j < it.nblk; ++j) {
+    const Half h0 = it.w.next();
+    const Half h1 = it.w.next();
+    const Half& hb = rc.kh ? h1 : h0;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint64_t valid = key_mask<kMask>(hb, rc, t);
+      if (!softmax_half<kMask>(p, sm, ss, tmem, rc, t, j, valid, m[t], l[t])) return false;
+    }
+  }
+  return true;
 }
 
 __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, uint32_t tmem, int warp, int lane) {
   volatile int* abort = &sm.abort;
   const long long budget = p.wait_budget;
   RowCtx rc;
-  rc.t = (warp - 4) >> 2;
-  rc.lane = lane;
-  const int t = rc.t;
   const int wq = warp & 3;
-  const int r = wq * 32 + lane;   // row inside the 128-row tile
-  rc.quarter = (t * 128 + r) >> 6;  // 64-row quarter of the 256-row item
-  const int quarter = rc.quarter;
-  const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-  rc.tS = tmem + lane_off + t * 256;
-  rc.tP = rc.tS + 128;
-  rc.tO = rc.tS + 192;
-  const uint32_t tO = rc.tO;
-  uint32_t sfull_c = 0, odone_c = 0;
+  rc.kh = (warp - 4) >> 2;
+  rc.r = wq * 32 + lane;
+  rc.lane = lane;
+  rc.lane_off = static_cast<uint32_t>(wq * 32) << 16;
+  const int r = rc.r;
+  SoftmaxState ss;
   bool ok = true;
 
   for (int item = blockIdx.x; ok && item < p.total_items; item += gridDim.x) {
     ItemInfo it = item_info(p, item);
     const HeadPlan& hp = p.heads[it.hi];
-    const int qrow = it.q0 + t * 128 + r;
-    float l = 0.f;
+    float m[2] = {-INFINITY, -INFINITY};  // running max of this key half, log2 units, per tile
+    float l[2] = {0.f, 0.f};              // running sum of this key half, per tile
     if (hp.kind == SAF3R_POSITION) {
-      // neighbour cells of this row's grid cell, as kept derived rows [lo, hi)
-      const bool patch_row = qrow < p.P * p.S && p.S > 1;
-      const int cell = patch_row ? qrow / p.S : 0;
-      const int qr = cell / p.gw, qc = cell - qr * p.gw;
-      const int R = hp.radius;
+      // neighbour cells of each tile row's grid cell, as kept derived rows [lo, hi)
 #pragma unroll
-      for (int x = 0; x < 2 * kMaxRadius + 1; ++x) {
-        const int dr = x - kMaxRadius;
-        const int rr = qr + dr;
-        const bool use = patch_row && dr >= -R && dr <= R && rr >= 0 && rr < p.gh;
-        const int ca = rr * p.gw + max(qc - R, 0);
-        const int cb = rr * p.gw + min(qc + R, p.gw - 1);
-        rc.nb_lo[x] = use ? hp.nb_base + ca * (p.S - 1) : 0;
-        rc.nb_hi[x] = use ? hp.nb_base + (cb + 1) * (p.S - 1) : 0;
+      for (int t = 0; t < 2; ++t) {
+        const int qrow = it.q0 + t * 128 + r;
+        const bool patch_row = qrow < p.P * p.S && p.S > 1;
+        const int cell = patch_row ? qrow / p.S : 0;
+        const int qr = cell / p.gw, qc = cell - qr * p.gw;
+        const int R = hp.radius;
+#pragma unroll
+        for (int x = 0; x < kNbIntervals; ++x) {
+          const int dr = x - kMaxRadius;
+          const int rr = qr + dr;
+          const bool use = patch_row && dr >= -R && dr <= R && rr >= 0 && rr < p.gh;
+          const int ca = rr * p.gw + max(qc - R, 0);
+          const int cb = rr * p.gw + min(qc + R, p.gw - 1);
+          rc.nb_lo[t][x] = use ? hp.nb_base + ca * (p.S - 1) : 0;
+          rc.nb_hi[t][x] = use ? hp.nb_base + (cb + 1) * (p.S - 1) : 0;
+        }
       }
-      ok = softmax_blocks<kMaskCells>(p, sm, it, rc, sfull_c, odone_c, l);
+      ok = softmax_blocks<kMaskCells>(p, sm, ss, tmem, it, rc, m, l);
     } else if (hp.kind == SAF3R_CORR) {
-      ok = softmax_blocks<kMaskTiles>(p, sm, it, rc, sfull_c, odone_c, l);
+      ok = softmax_blocks<kMaskTiles>(p, sm, ss, tmem, it, rc, m, l);
     } else {
-      ok = softmax_blocks<kMaskPlain>(p, sm, it, rc, sfull_c, odone_c, l);
+      ok = softmax_blocks<kMaskPlain>(p, sm, ss, tmem, it, rc, m, l);
     }
     if (!ok) break;
 
-    // epilogue: O / l of this row
-    if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], odone_c & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
+    // epilogue: merge the two key halves of each row; the warp of key half kh writes tile kh
+    const int t = rc.kh;
+    if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], ss.odone_c & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
       ok = false;
       break;
     }
-    ++odone_c;
+    ++ss.odone_c;
     tc_fence_after();
-    uint32_t o[2][32];
-    tmem_ld32(tO, o[0]);
-    tmem_ld32(tO + 32, o[1]);
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      sm.stats[rc.kh][tt][r][0] = m[tt];
+      sm.stats[rc.kh][tt][r][1] = l[tt];
+    }
+    // meet the other warp of these rows (bounded waits: a partner that gave up cannot hang this one)
+    mbar_arrive(&sm.pair[wq]);
+    if (!__all_sync(0xffffffffu, mbar_wait(&sm.pair[wq], ss.pair_c & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
+      ok = false;
+      break;
+    }
+    ++ss.pair_c;
+    const float ma = sm.stats[0][t][r][0], la = sm.stats[0][t][r][1];
+    const float mb = sm.stats[1][t][r][0], lb = sm.stats[1][t][r][1];
+    mbar_arrive(&sm.pair[wq]);  // stats may be overwritten by the next item once both warps are past this
+    if (!__all_sync(0xffffffffu, mbar_wait(&sm.pair[wq], ss.pair_c & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
+      ok = false;
+      break;
+    }
+    ++ss.pair_c;
+    const float mmax = fmaxf(ma, mb);
+    const float fa = ma == -INFINITY ? 0.f : fast_exp2(ma - mmax);
+    const float fb = mb == -INFINITY ? 0.f : fast_exp2(mb - mmax);
+    const float den = la * fa + lb * fb;
+    const float ia = den > 0.f ? fa / den : 0.f, ib = den > 0.f ? fb / den : 0.f;
+    uint32_t oa[2][32], ob[2][32];
+    const uint32_t tO = tmem + rc.lane_off + t * 256 + 128;
+    tmem_ld32(tO, oa[0]);
+    tmem_ld32(tO + 32, oa[1]);
+    tmem_ld32(tO + 64, ob[0]);
+    tmem_ld32(tO + 96, ob[1]);
     tmem_wait_ld();
     tc_fence_before();
+    float o[64];
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[c * 32 + i] = __uint_as_float(oa[c][i]) * ia + __uint_as_float(ob[c][i]) * ib;
+    const int qrow = it.q0 + t * 128 + r;
+    const int quarter = (t * 128 + r) >> 6;
     int token = -1;
     if (hp.q_src == 1) {
       if (qrow < p.N) token = position_token(p, qrow);
@@ -550,26 +578,17 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
       token = qrow;
     }
     if (token >= 0) {
-      const float inv = l > 0.f ? 1.f / l : 0.f;
       const long long rowoff = (static_cast<long long>(hp.head) * p.N + token) * kD;
       if (p.out_fp32) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + rowoff);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint32_t* w = &o[i >> 3][(4 * i) & 31];
-          dst[i] = make_float4(__uint_as_float(w[0]) * inv, __uint_as_float(w[1]) * inv,
-                               __uint_as_float(w[2]) * inv, __uint_as_float(w[3]) * inv);
-        }
+        for (int i = 0; i < 16; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
       } else {
         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + rowoff);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t* w = &o[i >> 2][(8 * i) & 31];
-          dst[i] = make_uint4(pack_bf16x2(__uint_as_float(w[0]) * inv, __uint_as_float(w[1]) * inv),
-                              pack_bf16x2(__uint_as_float(w[2]) * inv, __uint_as_float(w[3]) * inv),
-                              pack_bf16x2(__uint_as_float(w[4]) * inv, __uint_as_float(w[5]) * inv),
-                              pack_bf16x2(__uint_as_float(w[6]) * inv, __uint_as_float(w[7]) * inv));
-        }
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_uint4(pack_bf16x2(o[8 * i], o[8 * i + 1]), pack_bf16x2(o[8 * i + 2], o[8 * i + 3]),
+                              pack_bf16x2(o[8 * i + 4], o[8 * i + 5]), pack_bf16x2(o[8 * i + 6], o[8 * i + 7]));
       }
     }
   }
@@ -600,10 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.s_full[t], 1);
-      mbar_init(&sm.s_free[t], 4);
-      mbar_init(&sm.p_full[t], 4);
+      mbar_init(&sm.p_full[t], 8);
       mbar_init(&sm.o_done[t], 1);
     }
+    for (int w = 0; w < 4; ++w) mbar_init(&sm.pair[w], 64);
     sm.abort = 0;
     fence_mbar_init();
   }
