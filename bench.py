@@ -35,6 +35,44 @@ FLOP_PER_PAIR = 256  # q.k (2d) + p.v (2d), d = 64
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM traffic of one attention launch on this workload, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# source it was taken on: a changed kernel reports null until it is re-captured.
+# Taken on the S=32-view call (190,235,904 + 71,874,816 bytes) and scaled to the
+# S=100-view call by the token count (137,400 / 43,968): Q/K/V/O bytes grow with N.
+ATTN_TRAFFIC = {"kernel_source_sha256": "049d8a664072dafe70d6404b7196a28afd65d79ad24d86ce709c04479129fa96",
+                "bytes_per_launch": round((190235904 + 71874816) * 137400 / 43968), "workload": "s100"}
+
+
+def kernel_source_sha256():
+    import hashlib
+    with open(os.path.join(ROOT, "head_wise_dynamic_b200", "csrc", "attn_sm100.cu"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def attn_traffic(workload):
+    t = ATTN_TRAFFIC
+    if t["bytes_per_launch"] is None or t["workload"] != workload:
+        return None
+    return t["bytes_per_launch"] if t["kernel_source_sha256"] == kernel_source_sha256() else None
+
+
+def max_over_ranks(x, device):
+    """The largest value of x over all ranks (x itself with one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time (ms), per second."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -195,11 +233,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     hw.saf3r_check()
-    ms_step = t0.elapsed_time(t1) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step = float(tt.item())
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     call_ms = [a.elapsed_time(b) for a, b in ev_call]
     sel_ms = [a.elapsed_time(b) for a, b in ev_sel]
@@ -226,7 +260,7 @@ def run_ours(args):
     peak_key = "bf16_tflops_sustained" if timed_s > 1.0 else "bf16_tflops"
     peak = float(peaks[peak_key])
     achieved = pairs_call * FLOP_PER_PAIR / (attn_kernel_ms * 1e-3) / 1e12
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    value = job_throughput(flops_step, world, ms_step) / 1e12
 
     # end to end through the same API: pinned host inputs in, outputs back, every step
     e2e = None
@@ -257,12 +291,8 @@ def run_ours(args):
         b.record(stream)
         torch.cuda.synchronize()
         hw.saf3r_check()
-        e2e_ms = a.elapsed_time(b) / args.e2e_steps
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, dev)
+        e2e = {"value": job_throughput(flops_step, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
 
     cpu = None
@@ -285,7 +315,7 @@ def run_ours(args):
         "dense_ms": dense_ms, "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
         "speedup_vs_dense": dense_ms / statistics.mean(call_ms),
         "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": attn_traffic(args.workload),
                      "peak_source": f"{peak_src} {peak_key}",
                      "algorithmic": f"{pairs_call} kept pairs x 256 FLOP per launch"},
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clock_info,
@@ -308,14 +338,15 @@ def _blas_threads():
         return 1
 
 
-def cpu_baseline(wl, scene, qkv_call, pairs_call, budget_s=15.0, rows_per_head=None):
+def cpu_baseline(wl, scene, qkv_call, pairs_call, budget_s=15.0, chunk_rows=32):
     """The oracle, as it stands, on a bounded sample of the same workload.
 
-    Times the full index selection of one input and the sparse attention of a
-    few sampled rows per head, then extrapolates the rows to all N rows of the
-    4 layer calls: value = 4 * pairs * 256 / (t_select + 4 * t_rows * pairs / sampled_pairs)."""
+    Times the full index selection of one input, then the sparse attention of
+    uniformly drawn seeded rows (chunk_rows rows per head and chunk) until about budget_s
+    seconds of CPU work are spent, and extrapolates the rows to all N rows of the
+    layer calls: value = calls * pairs * 256 / (t_select + calls * t_rows * pairs / sampled_pairs)."""
     import oracle as O
-    from saf3r_synth import bf16_to_f32, sample_rows
+    from saf3r_synth import bf16_to_f32
 
     L = wl.layout
     Q, K, V = (bf16_to_f32(t) for t in qkv_call)
@@ -323,20 +354,25 @@ def cpu_baseline(wl, scene, qkv_call, pairs_call, budget_s=15.0, rows_per_head=N
     t = time.perf_counter()
     sel = O.select(L, wl.heads, Q, K, dino)
     t_sel = time.perf_counter() - t
-    rows_per_head = rows_per_head or 16
     sampled_pairs = 0
+    sampled_rows = 0
     t_rows = 0.0
-    for h, hc in enumerate(wl.heads):
-        rows = sample_rows(wl, h, rows_per_head, seed_extra=1)[:rows_per_head]
-        t = time.perf_counter()
-        O.sparse_rows(L, hc, sel, h, Q[h], K[h], V[h], rows)
-        t_rows += time.perf_counter() - t
-        sampled_pairs += sum(O.kept_count(L, hc, sel, h, int(i)) for i in rows)
+    chunk = 0
+    while chunk == 0 or t_sel + t_rows < budget_s:
+        for h, hc in enumerate(wl.heads):
+            rng = np.random.default_rng((wl.seed, 7, h, chunk))
+            rows = np.sort(rng.choice(L.N, size=min(chunk_rows, L.N), replace=False))
+            t = time.perf_counter()
+            O.sparse_rows(L, hc, sel, h, Q[h], K[h], V[h], rows)
+            t_rows += time.perf_counter() - t
+            sampled_pairs += sum(O.kept_count(L, hc, sel, h, int(i)) for i in rows)
+            sampled_rows += len(rows)
+        chunk += 1
     t_step = t_sel + wl.calls * t_rows * (pairs_call / sampled_pairs)
     return {"value": wl.calls * pairs_call * FLOP_PER_PAIR / t_step / 1e12, "unit": "TFLOP/s",
             "cores": _blas_threads(), "kind": "oracle",
             "sample": (f"full index selection of one input ({t_sel:.1f} s) + sparse attention of "
-                       f"{rows_per_head} sampled rows per head ({t_rows:.2f} s, {sampled_pairs} kept pairs), "
+                       f"{sampled_rows} seeded rows over {L.H} heads ({t_rows:.1f} s, {sampled_pairs} kept pairs), "
                        f"extrapolated to all {L.N} rows x {L.H} heads x {wl.calls} calls"),
             "seconds": t_sel + t_rows}
 
@@ -362,7 +398,7 @@ def run_reference(args):
     pairs_call = sum(O.kept_pairs(wl.layout, hc, sel, h) for h, hc in enumerate(wl.heads))
     vals, secs = [], []
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(wl, scene, calls, pairs_call, rows_per_head=4)
+        r = cpu_baseline(wl, scene, calls, pairs_call, budget_s=args.ref_seconds, chunk_rows=4)
         if i >= args.warmup:
             vals.append(r["value"])
             secs.append(r["seconds"])
@@ -391,6 +427,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=2.0, help="CPU seconds per reference-arm step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
