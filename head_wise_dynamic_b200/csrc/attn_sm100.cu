@@ -16,7 +16,8 @@
 //
 // Warp roles (12 warps, three warpgroups):
 //   warp 0      TMA producer: Q tiles, then K and V blocks into a 4-stage ring
-//   warp 1      MMA issuer (one thread): O_t += P_t V, then S_t = Q_t K^T of the next block
+//   warp 1      MMA issuer: O_t += P_t V, then S_t = Q_t K^T of the next block (the whole warp
+//               waits and computes descriptors, one elected lane issues)
 //   warps 2-3   idle (their registers go to the softmax warpgroups)
 //   warps 4-11  softmax: warp w owns rows 32*(w%4)..+31 of a tile (the TMEM lanes it may
 //               read) and key half (w-4)/4 of every 128-key block; all eight warps work
@@ -224,14 +225,16 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm,
     mbar_wait_drain(&sm.v_full[c % kStages], (c / kStages) & 1, drain);
 }
 
-// ------------------------------------------------------------------ MMA issuer (one thread)
+// ------------------------------------------------------------------ MMA issuer (one warp)
 //
 // For each key block and each tile in turn: O_t,a += P_t,a V[0:64] and O_t,b += P_t,b V[64:128]
 // once all eight softmax warps have written P_t, then S_t = Q_t K^T of the next block (it
-// overwrites P_t, which the products just issued have read: this thread's products execute
-// in issue order).  This thread sits on the critical path, so it does nothing but wait, add
-// descriptor offsets and issue; every product covers the whole block (keys a row does not
-// keep get P = 0).
+// overwrites P_t, which the products just issued have read: one lane issues every product,
+// and a lane's products execute in issue order).  The warp sits on the critical path, so it
+// does nothing but wait, add descriptor offsets and issue.  Running it converged (rather than
+// as a lone lane) keeps the descriptors warp-uniform, which measurably shortens the issue of
+// each 12-product tile step.  Every product covers the whole block (keys a row does not keep
+// get P = 0).
 struct MmaState {
   uint32_t pfull_c[2] = {0, 0};
 };
@@ -254,6 +257,8 @@ __device__ __forceinline__ void issue_qk(const Descs& d, uint32_t tmem, int t, u
   for (int kk = 0; kk < 4; ++kk) mma_ss(tmem + t * 256, dq + 2 * kk, dk + 2 * kk, idesc, kk > 0 ? 1u : 0u);
 }
 
+// Run by the whole warp: every lane waits and computes the (warp-uniform) descriptors, one
+// elected lane issues the products and their commits.
 __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint32_t tmem) {
   volatile int* abort = &sm.abort;
   const long long budget = p.wait_budget;
@@ -268,29 +273,33 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint
   bool ok = true;
   for (int item = blockIdx.x; ok && item < p.total_items; item += gridDim.x) {
     const int nblk = item_info(p, item).nblk;
-    if (!mbar_wait(&sm.q_full, items & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) break;
+    if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full, items & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) break;
     tc_fence_after();
     {
       const uint32_t stage = kv_c % kStages, ph = (kv_c / kStages) & 1;
-      if (!mbar_wait(&sm.k_full[stage], ph, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.k_full[stage], ph, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) break;
       tc_fence_after();
-      issue_qk(d, tmem, 0, stage);
-      mma_commit(&sm.s_full[0]);
-      issue_qk(d, tmem, 1, stage);
-      mma_commit(&sm.s_full[1]);
-      mma_commit(&sm.k_empty[stage]);
-      if (nblk == 1) mma_commit(&sm.q_empty);
+      if (elect_one()) {
+        issue_qk(d, tmem, 0, stage);
+        mma_commit(&sm.s_full[0]);
+        issue_qk(d, tmem, 1, stage);
+        mma_commit(&sm.s_full[1]);
+        mma_commit(&sm.k_empty[stage]);
+        if (nblk == 1) mma_commit(&sm.q_empty);
+      }
+      __syncwarp();
     }
     for (int j = 0; ok && j < nblk; ++j) {
       const uint32_t c = kv_c + j;
       const uint32_t cs = c % kStages, cph = (c / kStages) & 1;
       const bool has_next = j + 1 < nblk;
       const uint32_t ns = (c + 1) % kStages, nph = ((c + 1) / kStages) & 1;
-      if (has_next && !mbar_wait(&sm.k_full[ns], nph, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) {
+      if (has_next &&
+          !__all_sync(0xffffffffu, mbar_wait(&sm.k_full[ns], nph, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
         ok = false;
         break;
       }
-      if (!mbar_wait(&sm.v_full[cs], cph, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.v_full[cs], cph, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
         ok = false;
         break;
       }
@@ -298,33 +307,41 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint
       const uint64_t dv = d.v0 + cs * kStageDesc;
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if (!mbar_wait(&sm.p_full[t], st.pfull_c[t] & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&sm.p_full[t], st.pfull_c[t] & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
           ok = false;
           break;
         }
         ++st.pfull_c[t];
         tc_fence_after();
         const uint32_t s_col = tmem + t * 256, o_col = s_col + 128;
-        // key half a: P in S columns 0..31, keys 0..63 of V; key half b: S columns 64..95, keys 64..127
-        mma_ts(o_col, s_col, dv, idesc_pv, j > 0 ? 1u : 0u);
+        if (elect_one()) {
+          // key half a: P in S columns 0..31, keys 0..63 of V; key half b: S columns 64..95, keys 64..127
+          mma_ts(o_col, s_col, dv, idesc_pv, j > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < 4; ++kk) mma_ts(o_col, s_col + kk * 8, dv + 128 * kk, idesc_pv, 1u);
-        mma_ts(o_col + 64, s_col + 64, dv + 128 * 4, idesc_pv, j > 0 ? 1u : 0u);
+          for (int kk = 1; kk < 4; ++kk) mma_ts(o_col, s_col + kk * 8, dv + 128 * kk, idesc_pv, 1u);
+          mma_ts(o_col + 64, s_col + 64, dv + 128 * 4, idesc_pv, j > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < 4; ++kk) mma_ts(o_col + 64, s_col + 64 + kk * 8, dv + 128 * (4 + kk), idesc_pv, 1u);
-        if (has_next) {
-          issue_qk(d, tmem, t, ns);
-          mma_commit(&sm.s_full[t]);
-        } else {
-          mma_commit(&sm.o_done[t]);
+          for (int kk = 1; kk < 4; ++kk)
+            mma_ts(o_col + 64, s_col + 64 + kk * 8, dv + 128 * (4 + kk), idesc_pv, 1u);
+          if (has_next) {
+            issue_qk(d, tmem, t, ns);
+            mma_commit(&sm.s_full[t]);
+          } else {
+            mma_commit(&sm.o_done[t]);
+          }
         }
+        __syncwarp();
       }
       if (!ok) break;
-      mma_commit(&sm.v_empty[cs]);
-      if (has_next) {
-        mma_commit(&sm.k_empty[ns]);
-        if (j + 2 == nblk) mma_commit(&sm.q_empty);
+      if (elect_one()) {
+        mma_commit(&sm.v_empty[cs]);
+        if (has_next) {
+          mma_commit(&sm.k_empty[ns]);
+          if (j + 2 == nblk) mma_commit(&sm.q_empty);
+        }
       }
+      __syncwarp();
     }
     kv_c += nblk;
     ++items;
@@ -377,6 +394,7 @@ struct SoftmaxState {
   uint32_t pair_c = 0;
 };
 
+
 // One 64-key half-block of one tile for this thread's row: masks, running max, exponentials,
 // P (bf16) written over the half's first 32 S columns, arrival on p_full[t].
 template <int kMask>
@@ -388,6 +406,19 @@ __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, 
   ++ss.sfull_c[t];
   tc_fence_after();
   const uint32_t tS = tmem + rc.lane_off + t * 256 + rc.kh * 64;
+  if (kMask != kMaskPlain && __all_sync(0xffffffffu, valid == 0ull)) {
+    // no row of this warp keeps a key of this half-block: P = 0, the running max and sum stay
+    if (j == 0) m = -INFINITY;
+    uint32_t zero[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) zero[i] = 0u;
+    tmem_st32(tS, zero);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (rc.lane == 0) mbar_arrive(&sm.p_full[t]);
+    return true;
+  }
   float s[64];
   {
     uint32_t raw[2][32];
@@ -408,10 +439,8 @@ __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, 
 #pragma unroll
   for (int i = 0; i < 8; ++i) mp[i] = s[i];
 #pragma unroll
-  for (int i = 8; i < 64; ++i) mp[i & 7] = fmaxf(mp[i & 7], s[i]);
-  const float mx =
-      fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
-      kScaleLog2;
+  for (int i = 4; i < 32; ++i) mp[i & 7] = max3f(mp[i & 7], s[2 * i], s[2 * i + 1]);
+  const float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * kScaleLog2;
   float alpha = 1.f;
   bool rescale = false;
   if (j == 0) {
@@ -443,9 +472,10 @@ __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, 
   for (int i = 0; i < 8; ++i) rp[i] = 0.f;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    const float e0 = fast_exp2(fmaf(s[2 * i], kScaleLog2, -m_use));
-    const float e1 = fast_exp2(fmaf(s[2 * i + 1], kScaleLog2, -m_use));
-    rp[i & 7] += e0 + e1;
+    float x0 = s[2 * i], x1 = s[2 * i + 1];
+    ffma2(x0, x1, kScaleLog2, -m_use);
+    const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+    fadd2(rp[2 * (i & 3)], rp[2 * (i & 3) + 1], e0, e1);
     pk[i] = pack_bf16x2(e0, e1);
   }
   l = l * alpha + (((rp[0] + rp[1]) + (rp[2] + rp[3])) + ((rp[4] + rp[5]) + (rp[6] + rp[7])));
@@ -640,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) producer_role(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) mma_role(p, sm, tmem);
+    mma_role(p, sm, tmem);
     __syncwarp();
   } else if (warp >= 4) {
     reg_alloc_inc<200>();

@@ -218,4 +218,35 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// ---------------------------------------------------------------- warp and packed-f32 helpers
+// One lane of a converged warp (the lowest active one) gets true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}" : "=r"(pred));
+  return pred != 0;
+}
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+// (a, b) = (a, b) * s + (c, c), one packed instruction
+__device__ __forceinline__ void ffma2(float& a, float& b, float s, float c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f32x2(a, b)), "l"(f32x2(s, s)), "l"(f32x2(c, c)));
+  a = __uint_as_float(static_cast<uint32_t>(d));
+  b = __uint_as_float(static_cast<uint32_t>(d >> 32));
+}
+// (x, y) += (a, b), one packed instruction
+__device__ __forceinline__ void fadd2(float& x, float& y, float a, float b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f32x2(x, y)), "l"(f32x2(a, b)));
+  x = __uint_as_float(static_cast<uint32_t>(d));
+  y = __uint_as_float(static_cast<uint32_t>(d >> 32));
+}
+
 }  // namespace saf3r
