@@ -27,6 +27,11 @@
 // first 32 columns of its own key half once it has read them) and two accumulators
 // O_t,a / O_t,b (64 fp32 cols each), one per key half, merged with the halves' running
 // maxima and sums when the item ends.
+// The softmax warps never walk the key-run lists: a head with one implicit run (probe,
+// stride, dense) gets block j's half-blocks in closed form, and for list heads the producer,
+// which walks the list anyway, leaves each block's halves in shared memory next to its V
+// stage.  Warps whose 32 rows keep no key of a half-block (correspondence tiles of another
+// quarter, cells outside the neighbourhood) write P = 0 without computing anything.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -46,6 +51,14 @@ constexpr int kHalfBytes = 64 * 64 * 2;   // 64 rows x 64 bf16
 constexpr float kScaleLog2 = 0.18033688011112042f;  // log2(e) / sqrt(64)
 constexpr float kRescaleThreshold = 8.0f;           // log2 units: keep a stale max until it is 256x off
 
+// One 64-row half-block of keys.
+struct Half {
+  bool have;
+  Seg s;
+  int off;  // first row inside the run
+  int cnt;  // rows (<= 64)
+};
+
 struct AttnSmem {
   uint8_t q[2][kTileBytes];
   uint8_t k[kStages][kTileBytes];
@@ -53,18 +66,11 @@ struct AttnSmem {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_full[2], o_done[2];
+  Half info[kStages][2];      // the key halves of the block in each K/V stage (written by the producer)
   uint64_t pair[4];           // the two warps sharing rows 32*w..+31 (w = warp % 4) meet here at an item's end
   float stats[2][2][128][2];  // [key half][tile][row] = (running max, running sum) for the final merge
   uint32_t tmem_base;
   int abort;
-};
-
-// One 64-row half-block of keys.
-struct Half {
-  bool have;
-  Seg s;
-  int off;  // first row inside the run
-  int cnt;  // rows (<= 64)
 };
 
 // Iterates the 64-row half-blocks of one item's key runs.
@@ -209,6 +215,9 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm,
         ok = false;
         break;
       }
+      // the block's halves for the softmax warps; the arrival below releases them with the stage
+      sm.info[stage][0] = h0;
+      sm.info[stage][1] = h1;
       mbar_arrive_expect_tx(&sm.v_full[stage], kTileBytes);
       if (h0.have) load_half(hp, h0, sm.v[stage], &tmV, &tmVC, &sm.v_full[stage]); else tma_load_3d(sm.v[stage], &tmV, 0, -64, hp.head, &sm.v_full[stage]);
       if (h1.have) load_half(hp, h1, sm.v[stage] + kHalfBytes, &tmV, &tmVC, &sm.v_full[stage]); else tma_load_3d(sm.v[stage] + kHalfBytes, &tmV, 0, -64, hp.head, &sm.v_full[stage]);
@@ -389,11 +398,43 @@ __device__ __forceinline__ uint64_t key_mask(const Half& hb, const RowCtx& rc, i
 }
 
 struct SoftmaxState {
+  uint32_t kv_c = 0;  // key blocks seen (all items): the K/V stage and its phase
   uint32_t sfull_c[2] = {0, 0};
   uint32_t odone_c = 0;
   uint32_t pair_c = 0;
 };
 
+
+// O_t of this warp's key half (64 columns from tO) times alpha: the running max grew by more
+// than the threshold.  O_t already holds the previous blocks' products (s_full of this block
+// was committed after them).
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    uint32_t o[16];
+    tmem_ld16(tO + q * 16, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+    tmem_st16(tO + q * 16, o);
+  }
+}
+
+// P = 2^(s * scale - m) for the row's 64 logits as 32 bf16 pairs, and 8 partial row sums (a
+// single running sum would be a chain of dependent adds).
+__device__ __forceinline__ void exponentials(const float (&s)[64], float m, uint32_t (&pk)[32], float (&rp)[8]) {
+  const float m_use = (m == -INFINITY) ? 0.f : m;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) rp[i] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float x0 = s[2 * i], x1 = s[2 * i + 1];
+    ffma2(x0, x1, kScaleLog2, -m_use);
+    const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+    fadd2(rp[2 * (i & 3)], rp[2 * (i & 3) + 1], e0, e1);
+    pk[i] = pack_bf16x2(e0, e1);
+  }
+}
 
 // One 64-key half-block of one tile for this thread's row: masks, running max, exponentials,
 // P (bf16) written over the half's first 32 S columns, arrival on p_full[t].
@@ -435,48 +476,62 @@ __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, 
     for (int i = 0; i < 64; ++i)
       if (!((valid >> i) & 1ull)) s[i] = -INFINITY;
   }
-  float mp[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mp[i] = s[i];
-#pragma unroll
-  for (int i = 4; i < 32; ++i) mp[i & 7] = max3f(mp[i & 7], s[2 * i], s[2 * i + 1]);
-  const float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * kScaleLog2;
-  float alpha = 1.f;
-  bool rescale = false;
-  if (j == 0) {
-    m = mx;
-  } else if (mx > m + kRescaleThreshold) {
-    alpha = fast_exp2(m - mx);  // m may be -inf: alpha = 0
-    m = mx;
-    rescale = true;
-  }
-  if (__any_sync(0xffffffffu, rescale)) {
-    // rare: the running max grew by more than the threshold.  O_t of this half already holds the
-    // previous blocks' products (s_full of this block was committed after them); rescale it.
-    const uint32_t tO = tmem + rc.lane_off + t * 256 + 128 + rc.kh * 64;
-#pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
-      uint32_t o[16];
-      tmem_ld16(tO + q * 16, o);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-      tmem_st16(tO + q * 16, o);
-    }
-  }
-  const float m_use = (m == -INFINITY) ? 0.f : m;
-  // 8 independent partial row sums: a single running sum would be a chain of dependent adds
   uint32_t pk[32];
   float rp[8];
+  float alpha = 1.f;
+  if (kMask == kMaskPlain) {
+    // Probe, stride and dense heads: exponentials against the running max of the earlier
+    // blocks, with this block's max taken in the same pass; only on the first block, or when
+    // the max grew past the threshold, are they redone against the new max.
+    const float m_spec = (m == -INFINITY) ? 0.f : m;
+    float mp[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) rp[i] = 0.f;
+    for (int i = 0; i < 8; ++i) {
+      rp[i] = 0.f;
+      mp[i] = s[i];
+    }
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    float x0 = s[2 * i], x1 = s[2 * i + 1];
-    ffma2(x0, x1, kScaleLog2, -m_use);
-    const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-    fadd2(rp[2 * (i & 3)], rp[2 * (i & 3) + 1], e0, e1);
-    pk[i] = pack_bf16x2(e0, e1);
+    for (int i = 0; i < 32; ++i) {
+      float x0 = s[2 * i], x1 = s[2 * i + 1];
+      if (i >= 4) mp[i & 7] = max3f(mp[i & 7], x0, x1);
+      ffma2(x0, x1, kScaleLog2, -m_spec);
+      const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+      fadd2(rp[2 * (i & 3)], rp[2 * (i & 3) + 1], e0, e1);
+      pk[i] = pack_bf16x2(e0, e1);
+    }
+    const float mx =
+        max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * kScaleLog2;
+    const bool grow = (j == 0) || (mx > m + kRescaleThreshold);
+    if (__any_sync(0xffffffffu, grow)) {
+      const float m_new = grow ? mx : m;
+      if (j > 0) {
+        // rows whose max moved rescale O_t of this half (the others multiply by 1)
+        alpha = grow ? fast_exp2(m - m_new) : 1.f;  // m may be -inf: alpha = 0
+        rescale_o(tmem + rc.lane_off + t * 256 + 128 + rc.kh * 64, alpha);
+      }
+      m = m_new;
+      exponentials(s, m, pk, rp);
+    }
+  } else {
+    // Position and correspondence heads (whose masks move the max more often): the block's
+    // max first, then the exponentials.
+    float mp[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mp[i] = s[i];
+#pragma unroll
+    for (int i = 4; i < 32; ++i) mp[i & 7] = max3f(mp[i & 7], s[2 * i], s[2 * i + 1]);
+    const float mx =
+        max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * kScaleLog2;
+    bool rescale = false;
+    if (j == 0) {
+      m = mx;
+    } else if (mx > m + kRescaleThreshold) {
+      alpha = fast_exp2(m - mx);  // m may be -inf: alpha = 0
+      m = mx;
+      rescale = true;
+    }
+    if (__any_sync(0xffffffffu, rescale)) rescale_o(tmem + rc.lane_off + t * 256 + 128 + rc.kh * 64, alpha);
+    exponentials(s, m, pk, rp);
   }
   l = l * alpha + (((rp[0] + rp[1]) + (rp[2] + rp[3])) + ((rp[4] + rp[5]) + (rp[6] + rp[7])));
   tmem_st32(tS, pk);
@@ -492,15 +547,29 @@ template <int kMask>
 __device__ __forceinline__ bool softmax_blocks(const AttnParams& p, AttnSmem& sm, SoftmaxState& ss, uint32_t tmem,
                                                ItemInfo& it, const RowCtx& rc, float (&m)[2], float (&l)[2]) {
   for (int j = 0; j < it.nblk; ++j) {
-    const Half h0 = it.w.next();
-    const Half h1 = it.w.next();
-    const Half& hb = rc.kh ? h1 : h0;
+    Half hb;
+    if (kMask == kMaskPlain) {
+      // one implicit run: this warp's half-block of block j is a closed form
+      hb.s = it.w.implicit;
+      hb.off = (2 * j + rc.kh) * 64;
+      hb.have = hb.off < hb.s.len;
+      hb.cnt = min(64, hb.s.len - hb.off);
+    } else {
+      // the producer wrote this block's halves next to its V stage; that stage is not refilled
+      // before the products of this block, which wait for these warps
+      const uint32_t c = ss.kv_c + j, st = c % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.v_full[st], (c / kStages) & 1, &sm.abort, p.err, p.wait_budget,
+                                             SAF3R_ERR_TIMEOUT)))
+        return false;
+      hb = sm.info[st][rc.kh];
+    }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const uint64_t valid = key_mask<kMask>(hb, rc, t);
       if (!softmax_half<kMask>(p, sm, ss, tmem, rc, t, j, valid, m[t], l[t])) return false;
     }
   }
+  ss.kv_c += it.nblk;
   return true;
 }
 
