@@ -227,8 +227,98 @@ __global__ void __launch_bounds__(128) dino_pool_kernel(const float* __restrict_
   for (int c = threadIdx.x; c < dim; c += blockDim.x) tilevec[static_cast<size_t>(t) * dim + c] = mean[c] * inv;
 }
 
-// Cosines of R query tiles against all T tiles (fp64 dots of unit vectors,
-// rounded to fp32), then per query tile the kmax best tiles in rank order.
+// Inverse of order_key.
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// The warp's 8-bit-digit radix select over row[0..T): the key of the kmax-th largest value
+// and how many keys equal to it are taken.  Histogram counts are aggregated per warp
+// instruction (lanes that share a bin add once), so a narrow range of cosines, whose keys
+// share their high digits, does not serialise 32 lanes on one shared-memory counter.
+__device__ __forceinline__ void warp_radix_kth(const float* row, int T, int kmax, int* wh, int lane,
+                                               uint32_t& prefix, int& remaining) {
+  prefix = 0;
+  uint32_t mask = 0;
+  remaining = kmax;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) wh[i] = 0;
+    __syncwarp();
+    for (int v0 = 0; v0 < T; v0 += 32) {
+      const int v = v0 + lane;
+      uint32_t key = 0;
+      bool in = false;
+      if (v < T) {
+        key = order_key(row[v]);
+        in = (key & mask) == prefix;
+      }
+      const uint32_t act = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const uint32_t bin = (key >> shift) & 0xFFu;
+        const uint32_t peers = __match_any_sync(act, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&wh[bin], __popc(peers));
+      }
+    }
+    __syncwarp();
+    int b = 255, above = 0;
+    for (; b > 0; --b) {
+      if (above + wh[b] >= remaining) break;
+      above += wh[b];
+    }
+    prefix |= static_cast<uint32_t>(b) << shift;
+    remaining -= above;
+    mask |= 0xFFu << shift;
+    __syncwarp();
+  }
+}
+
+// The kmax largest values of row[0..T) (ties to the lower index) written to out[0..kmax) in
+// rank order (value descending, then index ascending).  One warp.
+__device__ __forceinline__ void warp_rank_row(const float* row, int T, int kmax, int* wh, int* widx, uint32_t* wkey,
+                                              int lane, int32_t* __restrict__ out) {
+  uint32_t prefix;
+  int remaining;
+  warp_radix_kth(row, T, kmax, wh, lane, prefix, remaining);
+  // gather the selected tiles in index order (lane-strided chunks keep the order)
+  int base = 0, eq_used = 0;
+  for (int v0 = 0; v0 < T; v0 += 32) {
+    const int v = v0 + lane;
+    uint32_t key = 0;
+    bool gt = false, eq = false;
+    if (v < T) {
+      key = order_key(row[v]);
+      gt = key > prefix;
+      eq = key == prefix;
+    }
+    const uint32_t eq_mask = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_used + __popc(eq_mask & ((1u << lane) - 1u));
+    const bool take = gt || (eq && eq_rank < remaining);
+    const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int pos = base + __popc(take_mask & ((1u << lane) - 1u));
+      widx[pos] = v;
+      wkey[pos] = key;
+    }
+    base += __popc(take_mask);
+    eq_used += __popc(eq_mask);
+  }
+  __syncwarp();
+  // rank order: by key descending, then tile index ascending
+  for (int i = lane; i < kmax; i += 32) {
+    const uint32_t ki = wkey[i];
+    const int vi = widx[i];
+    int rank = 0;
+    for (int j = 0; j < kmax; ++j) {
+      const uint32_t kj = wkey[j];
+      rank += (kj > ki) || (kj == ki && widx[j] < vi);
+    }
+    out[rank] = vi;
+  }
+  __syncwarp();
+}
+
+// Cosines of R query tiles against all T tiles (fp64 dots of unit vectors, rounded to
+// fp32), then per query tile the kmax best tiles in rank order.  General form, any dim.
 __global__ void __launch_bounds__(256) tile_topk_kernel(const float* __restrict__ tilevec, int T, int dim, int R,
                                                         int kmax, int32_t* __restrict__ ranked) {
   extern __shared__ uint8_t tk_smem[];
@@ -265,68 +355,134 @@ __global__ void __launch_bounds__(256) tile_topk_kernel(const float* __restrict_
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int* wh = hist + warp * 256;
-  int* widx = sel_idx + warp * kmax;
-  uint32_t* wkey = sel_key + warp * kmax;
-  for (int r = warp; r < nr; r += 8) {
-    const float* row = cs + static_cast<size_t>(r) * T;
-    uint32_t prefix = 0, mask = 0;
-    int remaining = kmax;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = lane; i < 256; i += 32) wh[i] = 0;
-      __syncwarp();
-      for (int v = lane; v < T; v += 32) {
-        const uint32_t key = order_key(row[v]);
-        if ((key & mask) == prefix) atomicAdd(&wh[(key >> shift) & 0xFF], 1);
-      }
-      __syncwarp();
-      int b = 255, above = 0;
-      for (; b > 0; --b) {
-        if (above + wh[b] >= remaining) break;
-        above += wh[b];
-      }
-      prefix |= static_cast<uint32_t>(b) << shift;
-      remaining -= above;
-      mask |= 0xFFu << shift;
-      __syncwarp();
+  for (int r = warp; r < nr; r += 8)
+    warp_rank_row(cs + static_cast<size_t>(r) * T, T, kmax, hist + warp * 256, sel_idx + warp * kmax,
+                  sel_key + warp * kmax, lane, ranked + static_cast<size_t>(u0 + r) * kmax);
+}
+
+// Fast form for dim <= 384 (kTkChunks float4 chunks of 128 features per lane).
+//
+// Eight query tiles per block, one per warp for the ranking.  Every lane keeps its slice of
+// the eight query vectors in registers; a warp takes one candidate tile v at a time with
+// coalesced loads, forms eight fp32 partial dots and folds them over the warp with a
+// transposing butterfly (after it, lane group (lane>>2)&7 holds row r's full dot).
+//
+// fp32 accumulation misses the fp64 dot by at most (12 + 5) * 2^-24 * sum|a_i b_i| <= 1.02e-6
+// (unit vectors: sum|a_i b_i| <= 1; 12 products per lane, 5 butterfly levels).  So every tile
+// of the exact top-kmax has an fp32 cosine >= (the fp32 kmax-th value) - 2.04e-6, and every
+// tile below (the fp32 kmax-th value) - kTkBand cannot reach it.  The ranking therefore
+// recomputes exactly (fp64 dot, rounded to fp32 as the general form does) every tile within
+// kTkBand of the fp32 kmax-th value, and ranks the row: the result is the general form's.
+constexpr int kTkRows = 8;
+constexpr int kTkChunks = 3;
+constexpr float kTkBand = 4e-6f;
+
+__device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+__global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __restrict__ tilevec, int T, int dim,
+                                                             int kmax, int32_t* __restrict__ ranked) {
+  extern __shared__ uint8_t tk_smem[];
+  float* cs = reinterpret_cast<float*>(tk_smem);                               // [8][T]
+  int* hist = reinterpret_cast<int*>(cs + static_cast<size_t>(kTkRows) * T);  // [8 warps][256]
+  int* sel_idx = hist + 8 * 256;                                               // [8 warps][kmax]
+  uint32_t* sel_key = reinterpret_cast<uint32_t*>(sel_idx + 8 * kmax);         // [8 warps][kmax]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u0 = blockIdx.x * kTkRows;
+  const int nr = min(kTkRows, T - u0);
+
+  float4 q[kTkRows][kTkChunks];
+#pragma unroll
+  for (int r = 0; r < kTkRows; ++r)
+#pragma unroll
+    for (int c = 0; c < kTkChunks; ++c) {
+      const int d = 128 * c + 4 * lane;
+      q[r][c] = (r < nr && d < dim) ? ld_f4(tilevec + static_cast<size_t>(u0 + r) * dim + d)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    // gather the selected tiles in index order (lane-strided chunks keep the order)
-    int base = 0, eq_used = 0;
-    for (int v0 = 0; v0 < T; v0 += 32) {
-      const int v = v0 + lane;
-      uint32_t key = 0;
-      bool gt = false, eq = false;
-      if (v < T) {
-        key = order_key(row[v]);
-        gt = key > prefix;
-        eq = key == prefix;
+  const int b2 = (lane >> 2) & 1, b3 = (lane >> 3) & 1, b4 = (lane >> 4) & 1;
+  const int my_row = (lane >> 2) & 7;
+  for (int v = warp; v < T; v += 8) {
+    const float* fv = tilevec + static_cast<size_t>(v) * dim;
+    float a[kTkRows];
+#pragma unroll
+    for (int r = 0; r < kTkRows; ++r) a[r] = 0.f;
+#pragma unroll
+    for (int c = 0; c < kTkChunks; ++c) {
+      const int d = 128 * c + 4 * lane;
+      if (d < dim) {
+        const float4 b = ld_f4(fv + d);
+#pragma unroll
+        for (int r = 0; r < kTkRows; ++r) {
+          a[r] = fmaf(q[r][c].x, b.x, a[r]);
+          a[r] = fmaf(q[r][c].y, b.y, a[r]);
+          a[r] = fmaf(q[r][c].z, b.z, a[r]);
+          a[r] = fmaf(q[r][c].w, b.w, a[r]);
+        }
       }
-      const uint32_t eq_mask = __ballot_sync(0xffffffffu, eq);
-      const int eq_rank = eq_used + __popc(eq_mask & ((1u << lane) - 1u));
-      const bool take = gt || (eq && eq_rank < remaining);
-      const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
-      if (take) {
-        const int pos = base + __popc(take_mask & ((1u << lane) - 1u));
-        widx[pos] = v;
-        wkey[pos] = key;
-      }
-      base += __popc(take_mask);
-      eq_used += __popc(eq_mask);
     }
-    __syncwarp();
-    // rank order: by key descending, then tile index ascending
-    for (int i = lane; i < kmax; i += 32) {
-      const uint32_t ki = wkey[i];
-      const int vi = widx[i];
-      int rank = 0;
-      for (int j = 0; j < kmax; ++j) {
-        const uint32_t kj = wkey[j];
-        rank += (kj > ki) || (kj == ki && widx[j] < vi);
-      }
-      ranked[static_cast<size_t>(u0 + r) * kmax + rank] = vi;
+    // transposing butterfly: 8 values per lane -> lane group g = (lane>>2)&7 holds row g's sum
+    float h4[4], h2[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float send = b4 ? a[i] : a[i + 4], keep = b4 ? a[i + 4] : a[i];
+      h4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
     }
-    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float send = b3 ? h4[i] : h4[i + 2], keep = b3 ? h4[i + 2] : h4[i];
+      h2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float h1;
+    {
+      const float send = b2 ? h2[0] : h2[1], keep = b2 ? h2[1] : h2[0];
+      h1 = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
+    h1 += __shfl_xor_sync(0xffffffffu, h1, 1);
+    if ((lane & 3) == 0 && my_row < nr) cs[static_cast<size_t>(my_row) * T + v] = h1;
   }
+  __syncthreads();
+  if (warp >= nr) return;
+  float* row = cs + static_cast<size_t>(warp) * T;
+  int* wh = hist + warp * 256;
+  uint32_t prefix;
+  int remaining;
+  warp_radix_kth(row, T, kmax, wh, lane, prefix, remaining);
+  const float thr = key_value(prefix) - kTkBand;
+  // exact values for every tile within the band: fp64 dot of this warp's query tile (the
+  // registers of row `warp`) with tile v, rounded to fp32
+  for (int v0 = 0; v0 < T; v0 += 32) {
+    const int v = v0 + lane;
+    uint32_t todo = __ballot_sync(0xffffffffu, v < T && row[v] >= thr);
+    while (todo) {
+      const int bit = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int w = v0 + bit;
+      const float* fv = tilevec + static_cast<size_t>(w) * dim;
+      double acc = 0.0;
+#pragma unroll
+      for (int c = 0; c < kTkChunks; ++c) {
+        const int d = 128 * c + 4 * lane;
+        if (d < dim) {
+          const float4 b = ld_f4(fv + d);
+          float4 qa = q[0][c];
+#pragma unroll
+          for (int r = 1; r < kTkRows; ++r)
+            if (r == warp) qa = q[r][c];
+          acc = fma(static_cast<double>(qa.x), static_cast<double>(b.x), acc);
+          acc = fma(static_cast<double>(qa.y), static_cast<double>(b.y), acc);
+          acc = fma(static_cast<double>(qa.z), static_cast<double>(b.z), acc);
+          acc = fma(static_cast<double>(qa.w), static_cast<double>(b.w), acc);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) row[w] = static_cast<float>(acc);
+    }
+  }
+  __syncwarp();
+  warp_rank_row(row, T, kmax, wh, sel_idx + warp * kmax, sel_key + warp * kmax, lane,
+                ranked + static_cast<size_t>(u0 + warp) * kmax);
 }
 
 // ---- query-tile grouping of the correspondence heads (a scheduling aid, cached with the indices)
@@ -513,15 +669,25 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
   if (sp.corr_kmax > 0) {
     const size_t pool_smem = sizeof(float) * 5 * sp.dim;
     dino_pool_kernel<<<sp.T, 128, pool_smem, stream>>>(dino, sp.N, sp.V, sp.ns, sp.P, sp.dim, tilevec);
-    const int R = tile_rows_per_block(sp.T, sp.dim, sp.corr_kmax);
-    if (R <= 0) return cudaErrorInvalidValue;
-    const size_t smem = sizeof(float) * (static_cast<size_t>(R) * sp.dim + static_cast<size_t>(R) * sp.T) +
-                        sizeof(int) * (8 * 256 + 16 * static_cast<size_t>(sp.corr_kmax));
-    cudaError_t e =
-        cudaFuncSetAttribute(tile_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    tile_topk_kernel<<<(sp.T + R - 1) / R, 256, smem, stream>>>(tilevec, sp.T, sp.dim, R, sp.corr_kmax,
-                                                                cache + sp.corr_off);
+    cudaError_t e = cudaSuccess;
+    const size_t fast_smem = sizeof(float) * static_cast<size_t>(kTkRows) * sp.T +
+                             sizeof(int) * (8 * 256 + 16 * static_cast<size_t>(sp.corr_kmax));
+    if (sp.dim <= 128 * kTkChunks && fast_smem <= 200 * 1024) {
+      e = cudaFuncSetAttribute(tile_topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(fast_smem));
+      if (e != cudaSuccess) return e;
+      tile_topk_fast_kernel<<<(sp.T + kTkRows - 1) / kTkRows, 256, fast_smem, stream>>>(
+          tilevec, sp.T, sp.dim, sp.corr_kmax, cache + sp.corr_off);
+    } else {
+      const int R = tile_rows_per_block(sp.T, sp.dim, sp.corr_kmax);
+      if (R <= 0) return cudaErrorInvalidValue;
+      const size_t smem = sizeof(float) * (static_cast<size_t>(R) * sp.dim + static_cast<size_t>(R) * sp.T) +
+                          sizeof(int) * (8 * 256 + 16 * static_cast<size_t>(sp.corr_kmax));
+      e = cudaFuncSetAttribute(tile_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      tile_topk_kernel<<<(sp.T + R - 1) / R, 256, smem, stream>>>(tilevec, sp.T, sp.dim, R, sp.corr_kmax,
+                                                                  cache + sp.corr_off);
+    }
     *n_launch += 2;
     // query-tile grouping for the attention work items
     size_t goff = static_cast<size_t>(reinterpret_cast<uint8_t*>(tilevec) - ws) +
