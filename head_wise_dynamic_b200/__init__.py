@@ -9,6 +9,7 @@ the compiled library and a B200.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from dataclasses import dataclass
 from typing import List, Optional, Sequence
@@ -77,6 +78,9 @@ def lib() -> ctypes.CDLL:
         L.saf3r_cache_export.restype = i32
         L.saf3r_kept_pairs.argtypes = [LP, CP, vp, ctypes.POINTER(ctypes.c_int64), vp]
         L.saf3r_kept_pairs.restype = i32
+        L.saf3r_choose_eq2.argtypes = [i32, i32, i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
+                                       i32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_double)]
+        L.saf3r_choose_eq2.restype = i32
         L.saf3r_set_kernel_events.argtypes = [vp, vp]
         L.saf3r_set_kernel_events.restype = None
         L.saf3r_check.argtypes = [vp]
@@ -215,6 +219,47 @@ def saf3r_profile_heads(layout, cand, q, k, v, dino, nmse_max, workspace, stream
                                    _stream(stream))
     _check(st, "saf3r_profile_heads")
     return chosen, nmse, pairs
+
+
+def saf3r_choose_eq2(nmse, pairs, base: int):
+    """The eq. 2 search (see include/saf3r.h) over per-input tables nmse [n_inputs][H][n_cand]
+    and pairs [n_inputs][H][n_cand]; returns (choice int32 [H], mean nmse [H][n_cand])."""
+    e = np.ascontiguousarray(nmse, dtype=np.float64)
+    w = np.ascontiguousarray(pairs, dtype=np.int64)
+    if e.ndim == 2:
+        e, w = e[None], w[None]
+    if e.ndim != 3 or e.shape != w.shape:
+        raise ValueError("nmse and pairs must be [n_inputs][H][n_cand] tables of one shape")
+    n_in, H, C = e.shape
+    choice = np.zeros(H, dtype=np.int32)
+    mean = np.zeros((H, C), dtype=np.float64)
+    dp = ctypes.POINTER(ctypes.c_double)
+    st = lib().saf3r_choose_eq2(n_in, H, C, e.ctypes.data_as(dp), w.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                int(base), choice.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), mean.ctypes.data_as(dp))
+    _check(st, "saf3r_choose_eq2")
+    return choice, mean
+
+
+def baseline_stride(sigma: float) -> int:
+    """Stride of the uniform-sampling baseline of sparsity at least sigma: ceil(1 / (1 - sigma))."""
+    if not 0.0 <= sigma < 1.0:
+        raise ValueError("sigma must be in [0, 1)")
+    return int(math.ceil(1.0 / (1.0 - sigma) - 1e-9))
+
+
+def profile_heads_eq2(layout, cand, base: int, inputs, workspace, stream=None):
+    """The eq. 2 search over a calibration set: saf3r_profile_heads on every input
+    (q, k, v, dino), then saf3r_choose_eq2 over the per-input tables.
+    Returns (choice int32 [H], mean nmse [H][n_cand], pairs [n_inputs][H][n_cand])."""
+    tables, costs = [], []
+    for q, k, v, dino in inputs:
+        _, nmse, pairs = saf3r_profile_heads(layout, cand, q, k, v, dino, 0.0, workspace, stream)
+        tables.append(nmse)
+        costs.append(pairs)
+    if not tables:
+        raise ValueError("the calibration set is empty")
+    choice, mean = saf3r_choose_eq2(np.stack(tables), np.stack(costs), base)
+    return choice, mean, np.stack(costs)
 
 
 def saf3r_cache_export(layout, cfg, cache, head: int, stream=None) -> np.ndarray:

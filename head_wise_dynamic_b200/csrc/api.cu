@@ -817,4 +817,34 @@ saf3r_status saf3r_profile_heads(const saf3r_layout* L, const saf3r_head_cfg* ca
   return SAF3R_OK;
 }
 
+saf3r_status saf3r_choose_eq2(int n_inputs, int H, int n_cand, const double* nmse, const int64_t* pairs,
+                              int base, int32_t* choice, double* nmse_mean) {
+  if (!nmse || !pairs || !choice || n_inputs < 1 || H < 1 || n_cand < 1 || base < 0 || base >= n_cand)
+    return SAF3R_ERR_INVALID;
+  const size_t per = static_cast<size_t>(H) * n_cand;
+  std::vector<double> e(per, 0.0), w(per, 0.0);
+  for (int i = 0; i < n_inputs; ++i)
+    for (size_t x = 0; x < per; ++x) {
+      e[x] += nmse[i * per + x];
+      w[x] += static_cast<double>(pairs[i * per + x]);
+    }
+  for (size_t x = 0; x < per; ++x) {
+    e[x] /= n_inputs;
+    w[x] /= n_inputs;
+  }
+  for (int h = 0; h < H; ++h) {
+    const double* eh = e.data() + static_cast<size_t>(h) * n_cand;
+    const double* wh = w.data() + static_cast<size_t>(h) * n_cand;
+    int cur = base;
+    for (int c = 0; c < n_cand; ++c) {
+      if (c == base) continue;
+      if (wh[c] <= wh[base] && eh[c] < eh[cur]) cur = c;
+    }
+    choice[h] = cur;
+  }
+  if (nmse_mean)
+    for (size_t x = 0; x < per; ++x) nmse_mean[x] = e[x];
+  return SAF3R_OK;
+}
+
 }  // extern "C"

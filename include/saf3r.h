@@ -183,6 +183,30 @@ saf3r_status saf3r_profile_heads(const saf3r_layout* layout, const saf3r_head_cf
                                  void* workspace, void* stream);
 
 /*
+ * The search of section 4.2, eq. 2 ("progressive local substitution"), as a
+ * host-side rule over the tables saf3r_profile_heads measured on each input
+ * of a calibration set.  Per head h and candidate c it averages eq. 1 over
+ * the n_inputs inputs (E[h][c], fp64 sum in input order / n_inputs) and the
+ * kept pairs likewise (W[h][c], the cost: Omega = 4*d*pairs, so comparisons of
+ * pairs are comparisons of Omega).  Then, per head, it starts from the
+ * baseline candidate `base` (the uniform-stride SCAN candidate at the target
+ * sparsity sigma: stride ceil(1 / (1 - sigma))) and visits the other
+ * candidates in index order, making c the current choice when
+ * W[h][c] <= W[h][base] and E[h][c] < E[h][current].  The result minimises the
+ * error under the baseline's cost; ties go to the baseline, then to the lower
+ * candidate index.
+ *
+ * nmse:  HOST double  [n_inputs][H][n_cand] (saf3r_profile_heads' nmse, per input)
+ * pairs: HOST int64   [n_inputs][H][n_cand] (saf3r_profile_heads' pairs, per input)
+ * choice: HOST int32  [H] out, the chosen candidate index per head
+ * nmse_mean: HOST double [H][n_cand] out (E), or NULL
+ * Returns SAF3R_ERR_INVALID for null inputs, n_inputs, H or n_cand < 1, or
+ * base out of range.  No device work, no stream.
+ */
+saf3r_status saf3r_choose_eq2(int n_inputs, int H, int n_cand, const double* nmse, const int64_t* pairs,
+                              int base, int32_t* choice, double* nmse_mean);
+
+/*
  * Copy one head's cached index list to host memory (synchronizes `stream`):
  * PROBE head -> its k kept patch keys (ascending); CORR head -> the ranked
  * tile list int32 [T][k] truncated to that head's k.  *n receives the number

@@ -326,6 +326,34 @@ def choose_config(nmse_row: Sequence[float], omega_row: Sequence[int], nmse_max:
     return min(range(len(nmse_row)), key=lambda c: (nmse_row[c], c))
 
 
+def baseline_stride(sigma: float) -> int:
+    """Stride of the uniform-sampling baseline with sparsity at least sigma (section 4.2 starts
+    the search from uniform sampling at sparsity ratio sigma; section 5.1 uses sigma = 0.85):
+    keeping one key in s gives sparsity 1 - 1/s >= sigma for s = ceil(1 / (1 - sigma))."""
+    s = 1
+    while 1.0 - 1.0 / s < sigma - 1e-12:
+        s += 1
+    return s
+
+
+def choose_eq2(nmse_tables, pairs_tables, base: int) -> List[int]:
+    """Section 4.2, eq. 2 by progressive substitution: eq. 1 averaged over the calibration
+    inputs, cost Omega = 4*d*mean(kept pairs).  Per head, start from the baseline candidate;
+    walk the candidates in order and substitute c whenever it costs no more than the
+    baseline and its averaged NMSE is lower than the current choice's."""
+    E = np.mean(np.asarray(nmse_tables, dtype=np.float64), axis=0)
+    W = np.mean(np.asarray(pairs_tables, dtype=np.float64), axis=0)
+    H, C = E.shape
+    out = []
+    for h in range(H):
+        cur = base
+        for c in range(C):
+            if c != base and W[h, c] <= W[h, base] and E[h, c] < E[h, cur]:
+                cur = c
+        out.append(cur)
+    return out
+
+
 def apply_candidate(hc, h: int):
     """A candidate applied to head h: scan candidates take phase = h mod stride."""
     if hc.kind == SCAN:

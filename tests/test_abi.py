@@ -2,6 +2,7 @@
 rejects bad arguments on the host (no GPU needed: no compute call is made)."""
 import ctypes
 
+import numpy as np
 import pytest
 
 import head_wise_dynamic_b200 as hw
@@ -65,3 +66,27 @@ def test_calls_reject_bad_arguments_before_any_launch():
     L.d = 128
     assert lib.saf3r_dense_attn(ctypes.byref(L), 0x1000, 0x1000, 0x1000, 0x1000, 0, 0x1000, None) == \
         hw.ERR_UNSUPPORTED
+
+
+def test_choose_eq2_host_rule_matches_oracle():
+    """saf3r_choose_eq2 is host logic: the C rule against the oracle on random tables."""
+    import oracle as O
+    rng = np.random.default_rng(11)
+    for _ in range(100):
+        n_in, H, C = int(rng.integers(1, 4)), int(rng.integers(1, 6)), int(rng.integers(1, 9))
+        E = rng.choice([0.01, 0.02, 0.05, 0.1], size=(n_in, H, C)) * rng.choice([1.0, 1.5], size=(n_in, H, C))
+        W = rng.integers(1, 6, size=(n_in, H, C)).astype(np.int64) * 1000
+        base = int(rng.integers(0, C))
+        choice, mean = hw.saf3r_choose_eq2(E, W, base)
+        assert choice.tolist() == O.choose_eq2(E, W, base)
+        assert np.allclose(mean, E.mean(axis=0), rtol=0, atol=1e-15)
+
+
+def test_choose_eq2_rejects_bad_arguments():
+    E = np.zeros((1, 2, 3))
+    W = np.zeros((1, 2, 3), dtype=np.int64)
+    with pytest.raises(hw.Saf3rError):
+        hw.saf3r_choose_eq2(E, W, 3)
+    with pytest.raises(hw.Saf3rError):
+        hw.saf3r_choose_eq2(E, W, -1)
+    assert hw.baseline_stride(0.85) == 7

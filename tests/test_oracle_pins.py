@@ -252,3 +252,52 @@ def test_kept_pairs_and_omega():
     pairs = O.kept_pairs(L, HeadCfg(SCAN, stride=3, phase=1), sel, 0)
     assert pairs == L.N * len(O.stride_set(L, 3, 1))
     assert O.omega(L, pairs) == 256 * pairs
+
+
+def test_baseline_stride():
+    # keeping one key in s is sparsity 1 - 1/s; the smallest s reaching sigma
+    assert O.baseline_stride(0.85) == 7        # 1 - 1/7 = 0.857 >= 0.85 > 1 - 1/6
+    assert O.baseline_stride(0.75) == 4
+    assert O.baseline_stride(0.0) == 1
+    for sigma in np.linspace(0.0, 0.95, 40):
+        s = O.baseline_stride(float(sigma))
+        assert 1 - 1 / s >= sigma - 1e-12 and (s == 1 or 1 - 1 / (s - 1) < sigma)
+
+
+def _eq2_brute(E, W, base):
+    """eq. 2 restated as a constrained argmin: least error among the candidates that cost no
+    more than the baseline; ties to the baseline, then to the lower index."""
+    H, C = E.shape
+    out = []
+    for h in range(H):
+        feas = [c for c in range(C) if W[h, c] <= W[h, base]]
+        out.append(min(feas, key=lambda c: (E[h, c], 0 if c == base else 1, c)))
+    return out
+
+
+def test_choose_eq2_rule():
+    # head 0: candidate 1 is cheaper and better; 2 is better still but costs more than the baseline
+    # head 1: nothing under the baseline cost beats it -> the baseline stays
+    # head 2: equal error to the baseline -> the baseline stays
+    E = np.array([[0.5, 0.4, 0.1, 0.45], [0.2, 0.3, 0.25, 0.1], [0.3, 0.3, 0.3, 0.3]])
+    W = np.array([[100, 90, 120, 80], [100, 60, 100, 101], [100, 50, 50, 50]])
+    assert O.choose_eq2([E], [W], 0) == [1, 0, 0]
+    # averaging over inputs: the second input flips head 0's order of 1 and 3
+    E2 = E.copy()
+    E2[0] = [0.5, 0.6, 0.1, 0.2]
+    assert O.choose_eq2([E, E2], [W, W], 0) == [3, 0, 0]
+
+
+def test_choose_eq2_equals_constrained_argmin():
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        H, C = int(rng.integers(1, 5)), int(rng.integers(1, 8))
+        n_in = int(rng.integers(1, 4))
+        Es = rng.choice([0.1, 0.2, 0.3, 0.4], size=(n_in, H, C))    # coarse values: many ties
+        Ws = rng.integers(1, 5, size=(n_in, H, C)) * 10
+        base = int(rng.integers(0, C))
+        got = O.choose_eq2(Es, Ws, base)
+        assert got == _eq2_brute(Es.mean(axis=0), Ws.mean(axis=0), base)
+        E, W = Es.mean(axis=0), Ws.mean(axis=0)
+        for h, c in enumerate(got):
+            assert W[h, c] <= W[h, base] and E[h, c] <= E[h, base]
