@@ -24,7 +24,7 @@ def test_eq2_search_matches_oracle():
     scene = Scene(wl)
     dino_np = scene.dino()
     dino = torch.from_numpy(dino_np).cuda()
-    inputs = [qkv(scene, layer, device="cuda") + (dino,) for layer in range(2)]
+    inputs = [tuple(qkv(scene, layer, device="cuda")) + (dino,) for layer in range(2)]
     Lc = hw.layout_of(L)
     ws = torch.empty(hw.saf3r_profile_workspace_bytes(Lc, cands), dtype=torch.uint8, device="cuda")
     choice, mean, pairs = hw.profile_heads_eq2(Lc, cands, 0, inputs, ws)
