@@ -141,22 +141,9 @@ __global__ void __launch_bounds__(1024) probe_topk_kernel(const float* __restric
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    // lanes that share a bin add once per warp instruction: scores concentrate in a few
-    // high-digit bins, and per-lane atomics on one counter would serialise the warp
-    for (int j0 = 0; j0 < N; j0 += blockDim.x) {
-      const int j = j0 + static_cast<int>(threadIdx.x);
-      uint32_t key = 0;
-      bool in = false;
-      if (j < N) {
-        key = order_key(sc[j]);
-        in = (key & mask) == prefix;
-      }
-      const uint32_t act = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const uint32_t bin = (key >> shift) & 0xFFu;
-        const uint32_t peers = __match_any_sync(act, bin);
-        if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
-      }
+    for (int j = threadIdx.x; j < N; j += blockDim.x) {
+      const uint32_t key = order_key(sc[j]);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
