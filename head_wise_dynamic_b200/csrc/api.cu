@@ -138,6 +138,10 @@ saf3r_status check_cfg(const Dims& d, const saf3r_head_cfg* cfg, int H) {
       case SAF3R_SCAN:
         if (c.stride < 1 || c.phase < 0 || c.phase >= c.stride || c.phase >= d.N) return SAF3R_ERR_INVALID;
         break;
+      case SAF3R_HYBRID:
+        if (c.k < 1 || c.k > d.T || d.V < kTile + d.ns) return SAF3R_ERR_INVALID;
+        if (c.stride < 1 || c.phase < 0 || c.phase >= c.stride || c.phase >= d.N) return SAF3R_ERR_INVALID;
+        break;
       case SAF3R_DENSE:
         break;
       default:
@@ -161,7 +165,7 @@ uint64_t cache_hash(const saf3r_layout* L, const saf3r_head_cfg* cfg) {
   uint64_t h = 1469598103934665603ull;
   h = fnv1a(h, L, sizeof(saf3r_layout));
   for (int i = 0; i < L->H; ++i) {
-    const int32_t v[2] = {cfg[i].type, (cfg[i].type == SAF3R_PROBE || cfg[i].type == SAF3R_CORR) ? cfg[i].k : 0};
+    const int32_t v[2] = {cfg[i].type, (cfg[i].type == SAF3R_PROBE || tile_kind(cfg[i].type)) ? cfg[i].k : 0};
     h = fnv1a(h, v, sizeof(v));
   }
   return h;
@@ -185,7 +189,7 @@ CacheLayout cache_layout(const Dims& d, const saf3r_head_cfg* cfg) {
       c.probe_off[h] = static_cast<int>(ints);
       ints += (cfg[h].k + 63) & ~63;
     }
-    if (cfg[h].type == SAF3R_CORR) c.corr_kmax = std::max(c.corr_kmax, cfg[h].k);
+    if (tile_kind(cfg[h].type)) c.corr_kmax = std::max(c.corr_kmax, cfg[h].k);
   }
   c.corr_off = static_cast<int>(ints);
   ints += static_cast<size_t>(d.T) * c.corr_kmax;
@@ -203,7 +207,7 @@ struct SparseLayout {
   std::vector<int> kc_begin, n_rows, qc_begin, n_lat, n_off, off_list;
   // shared plan lists
   struct List {
-    int kind, param, cap, n_items;
+    int kind, param, tail, cap, n_items;  // tail: rows of the derived run that ends every item (tile lists)
     long long seg_begin, cnt_begin;
   };
   std::vector<List> lists;
@@ -241,7 +245,8 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
       case SAF3R_PROBE:
         rows = nsp + c.k;
         break;
-      case SAF3R_SCAN: {
+      case SAF3R_SCAN:
+      case SAF3R_HYBRID: {  // the lattice, then the specials off it
         s.n_lat[h] = (d.N - c.phase + c.stride - 1) / c.stride;
         int off = 0;
         for (int sv = 0; sv < d.S; ++sv)
@@ -262,15 +267,21 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
     s.kc_begin[h] = static_cast<int>(s.kc_rows);
     s.n_rows[h] = rows;
     s.kc_rows += rows;
-    if (c.type == SAF3R_POSITION || c.type == SAF3R_CORR) {
+    if (c.type == SAF3R_POSITION || tile_kind(c.type)) {
+      // tile heads share a list when their budget and derived-run length agree (the lattice
+      // masks of a hybrid head are applied in the kernel, not stored in the list)
+      const int kind = c.type == SAF3R_POSITION ? SAF3R_POSITION : SAF3R_CORR;
       const int param = c.type == SAF3R_POSITION ? c.radius : c.k;
+      const int tail = c.type == SAF3R_POSITION ? 0 : rows;
       int found = -1;
       for (size_t i = 0; i < s.lists.size(); ++i)
-        if (s.lists[i].kind == c.type && s.lists[i].param == param) found = static_cast<int>(i);
+        if (s.lists[i].kind == kind && s.lists[i].param == param && s.lists[i].tail == tail)
+          found = static_cast<int>(i);
       if (found < 0) {
         SparseLayout::List l;
-        l.kind = c.type;
+        l.kind = kind;
         l.param = param;
+        l.tail = tail;
         l.n_items = c.type == SAF3R_POSITION ? items_of(d.N) : (d.T + 3) / 4;
         l.cap = c.type == SAF3R_POSITION ? position_cap(d, c.radius) : 4 * c.k + 1;
         l.seg_begin = s.seg_total;
@@ -311,6 +322,8 @@ double est_keys(const Dims& d, const saf3r_head_cfg& c, const SparseLayout& s, i
       return s.n_rows[h];
     case SAF3R_CORR:
       return 1.5 * kTile * c.k + d.ns * d.S;
+    case SAF3R_HYBRID:
+      return 1.5 * kTile * c.k + s.n_rows[h];
     default:
       return d.N;
   }
@@ -369,7 +382,7 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     x.n_lat = s.n_lat[h];
     x.probe_off = cl.probe_off[h];
     x.off_list = s.off_list[h];
-    any_scan |= cfg[h].type == SAF3R_SCAN;
+    any_scan |= lattice_kind(cfg[h].type);
   }
   da.kc_total = s.kc_rows;
   da.qc_total = s.qc_rows;
@@ -386,8 +399,8 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
                                             segs + l.seg_begin, cnts + l.cnt_begin, stream));
     } else {
       st = cuda_status(launch_plan_corr(cache_i + cl.corr_off, cache_i + cl.order_off, cl.corr_kmax, l.param, d.T,
-                                        d.N, d.V, d.ns, d.S, segs + l.seg_begin, l.cap, cnts + l.cnt_begin, dev.err,
-                                        stream));
+                                        d.N, d.V, d.ns, l.tail, segs + l.seg_begin, l.cap, cnts + l.cnt_begin,
+                                        dev.err, stream));
     }
     ++launches;
     if (st != SAF3R_OK) return st;
@@ -407,8 +420,10 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     HeadPlan& hp = p.heads[i];
     hp.head = h;
     hp.kind = c.type;
-    hp.q_src = c.type == SAF3R_POSITION ? 1 : (c.type == SAF3R_CORR ? 2 : 0);
-    hp.q_base = c.type == SAF3R_CORR ? cl.order_off : (s.qc_begin[h] < 0 ? 0 : s.qc_begin[h]);
+    hp.q_src = c.type == SAF3R_POSITION ? 1 : (tile_kind(c.type) ? 2 : 0);
+    hp.q_base = tile_kind(c.type) ? cl.order_off : (s.qc_begin[h] < 0 ? 0 : s.qc_begin[h]);
+    hp.lat_stride = c.type == SAF3R_HYBRID ? c.stride : 0;
+    hp.lat_phase = c.type == SAF3R_HYBRID ? c.phase : 0;
     hp.kc_base = s.kc_begin[h];
     hp.n_items = items_of(d.N);
     hp.item_begin = item;
@@ -508,7 +523,7 @@ size_t saf3r_workspace_bytes(const saf3r_layout* L, const saf3r_head_cfg* cfg, i
     bool corr = false;
     for (int h = 0; h < d.H; ++h) {
       n_probe += cfg[h].type == SAF3R_PROBE;
-      corr |= cfg[h].type == SAF3R_CORR;
+      corr |= tile_kind(cfg[h].type);
     }
     return select_workspace_bytes(n_probe, d.N, d.T, d.dino_dim, corr);
   }
@@ -524,7 +539,7 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   const Dims d = make_dims(*L);
   if ((st = check_cfg(d, cfg, L->H)) != SAF3R_OK) return st;
   bool corr = false;
-  for (int h = 0; h < d.H; ++h) corr |= cfg[h].type == SAF3R_CORR;
+  for (int h = 0; h < d.H; ++h) corr |= tile_kind(cfg[h].type);
   if (!q || !k || !cache || !workspace || !aligned16(q) || !aligned16(k) || !aligned16(cache) ||
       !aligned16(workspace) || (corr && (!dino || !aligned16(dino))))
     return SAF3R_ERR_INVALID;
@@ -622,7 +637,7 @@ saf3r_status saf3r_cache_export(const saf3r_layout* L, const saf3r_head_cfg* cfg
       return SAF3R_ERR_CUDA;
     return SAF3R_OK;
   }
-  if (c.type == SAF3R_CORR) {
+  if (tile_kind(c.type)) {
     *n = static_cast<size_t>(d.T) * c.k;
     if (!host_idx) return SAF3R_OK;
     std::vector<int32_t> all(static_cast<size_t>(d.T) * cl.corr_kmax);
@@ -640,7 +655,7 @@ saf3r_status saf3r_cache_export(const saf3r_layout* L, const saf3r_head_cfg* cfg
 
 static saf3r_head_cfg apply_candidate(const saf3r_head_cfg& c, int h) {
   saf3r_head_cfg r = c;
-  if (c.type == SAF3R_SCAN) r.phase = h % c.stride;
+  if (lattice_kind(c.type)) r.phase = h % c.stride;
   return r;
 }
 
@@ -688,15 +703,26 @@ static long long pairs_of(const Dims& d, const saf3r_head_cfg& c, const std::vec
         }
       return tot;
     }
-    case SAF3R_CORR: {
+    case SAF3R_CORR:
+    case SAF3R_HYBRID: {
+      // specials (and the lattice), then the patch tokens of the kept tiles not already counted
+      const bool lat = c.type == SAF3R_HYBRID;
+      long long base = nsp;
+      if (lat) {
+        base = (N - c.phase + c.stride - 1) / c.stride;
+        for (int sv = 0; sv < d.S; ++sv)
+          for (int i = 0; i < d.ns; ++i)
+            if (((static_cast<long long>(sv) * d.V + i) % c.stride) != c.phase) ++base;
+      }
       long long tot = 0;
       for (int u = 0; u < d.T; ++u) {
         const long long rows = std::min<long long>(kTile, N - static_cast<long long>(u) * kTile);
-        long long keys = nsp;
+        long long keys = base;
         for (int r = 0; r < c.k; ++r) {
           const long long v = ranked[static_cast<size_t>(u) * kmax + r];
           const long long t0 = v * kTile, t1 = std::min(N, t0 + kTile);
-          for (long long t = t0; t < t1; ++t) keys += (t % d.V) >= d.ns;
+          for (long long t = t0; t < t1; ++t)
+            keys += (t % d.V) >= d.ns && !(lat && t % c.stride == c.phase);
         }
         tot += rows * keys;
       }
@@ -741,7 +767,7 @@ saf3r_status saf3r_profile_heads(const saf3r_layout* L, const saf3r_head_cfg* ca
   for (int c = 0; c < n_cand; ++c) {
     for (int h = 0; h < d.H; ++h) cfg[h] = apply_candidate(cand[c], h);
     if ((st = check_cfg(d, cfg.data(), d.H)) != SAF3R_OK) return st;
-    any_corr |= cand[c].type == SAF3R_CORR;
+    any_corr |= tile_kind(cand[c].type);
   }
   if (any_corr && !dino) return SAF3R_ERR_INVALID;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -769,7 +795,7 @@ saf3r_status saf3r_profile_heads(const saf3r_layout* L, const saf3r_head_cfg* ca
     for (int h = 0; h < d.H; ++h) cfg[h] = apply_candidate(cand[c], h);
     if ((st = saf3r_select_kv(L, cfg.data(), q, k, dino, cache, inner, stream)) != SAF3R_OK) return st;
     launches += t_launches;
-    if (cand[c].type == SAF3R_CORR) {
+    if (tile_kind(cand[c].type)) {
       const CacheLayout cl = cache_layout(d, cfg.data());
       kmax[c] = cl.corr_kmax;
       ranked[c].resize(static_cast<size_t>(d.T) * cl.corr_kmax);
@@ -783,7 +809,7 @@ saf3r_status saf3r_profile_heads(const saf3r_layout* L, const saf3r_head_cfg* ca
                                 sums + static_cast<size_t>(c) * d.H * 2, s)) != SAF3R_OK)
       return SAF3R_ERR_CUDA;
     launches += 2;
-    if (cand[c].type == SAF3R_CORR && cudaStreamSynchronize(s) != cudaSuccess) return SAF3R_ERR_CUDA;
+    if (tile_kind(cand[c].type) && cudaStreamSynchronize(s) != cudaSuccess) return SAF3R_ERR_CUDA;
   }
   std::vector<double> hs(static_cast<size_t>(n_cand) * d.H * 2);
   if (cudaMemcpyAsync(hs.data(), sums, hs.size() * sizeof(double), cudaMemcpyDeviceToHost, s) != cudaSuccess ||

@@ -374,7 +374,18 @@ struct RowCtx {
   int lane;
   uint32_t lane_off; // TMEM lane field of this warp
   int nb_lo[2][kNbIntervals], nb_hi[2][kNbIntervals];  // position heads: kept derived rows [lo, hi) per tile
+  int lat_stride, lat_phase;  // hybrid heads: the lattice (counted in the derived run), 0 = none
 };
+
+// Bits b of a 64-key half-block starting at token j0 whose token j0 + b lies on the lattice
+// j = phase (mod stride).
+__device__ __forceinline__ uint64_t lattice_bits(int j0, int stride, int phase) {
+  int b = (phase - j0) % stride;
+  if (b < 0) b += stride;
+  uint64_t m = 0ull;
+  for (; b < 64; b += stride) m |= 1ull << b;
+  return m;
+}
 
 template <int kMask>
 __device__ __forceinline__ uint64_t key_mask(const Half& hb, const RowCtx& rc, int t) {
@@ -385,6 +396,8 @@ __device__ __forceinline__ uint64_t key_mask(const Half& hb, const RowCtx& rc, i
   if (kMask == kMaskTiles) {
     const int lo = (hb.s.flags >> 8) & 0xFF, hi = (hb.s.flags >> 16) & 0xFF;
     if (hi > lo) v &= ~range_bits(max(lo - hb.off, 0), min(hi - hb.off, 64));
+    // a hybrid head's lattice keys inside a tile are already counted in its derived run
+    if (rc.lat_stride > 0 && hb.s.src == 0) v &= ~lattice_bits(hb.s.row0 + hb.off, rc.lat_stride, rc.lat_phase);
   }
   if (kMask == kMaskCells && (hb.s.flags & kSegCellMask)) {
     const int base = hb.s.row0 + hb.off;
@@ -612,7 +625,9 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
         }
       }
       ok = softmax_blocks<kMaskCells>(p, sm, ss, tmem, it, rc, m, l);
-    } else if (hp.kind == SAF3R_CORR) {
+    } else if (hp.kind == SAF3R_CORR || hp.kind == SAF3R_HYBRID) {
+      rc.lat_stride = hp.lat_stride;
+      rc.lat_phase = hp.lat_phase;
       ok = softmax_blocks<kMaskTiles>(p, sm, ss, tmem, it, rc, m, l);
     } else {
       ok = softmax_blocks<kMaskPlain>(p, sm, ss, tmem, it, rc, m, l);

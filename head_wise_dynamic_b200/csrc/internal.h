@@ -14,6 +14,11 @@ constexpr int kMaxRadius = 3;
 constexpr uint32_t kCacheMagic = 0x52334653u;  // "SF3R"
 constexpr uint32_t kCacheVersion = 1;
 
+// Heads whose keys include ranked DINO tiles (they share the cached tile lists), and heads
+// whose keys include the stride lattice (they get the lattice as derived rows).
+__host__ __device__ inline bool tile_kind(int type) { return type == SAF3R_CORR || type == SAF3R_HYBRID; }
+__host__ __device__ inline bool lattice_kind(int type) { return type == SAF3R_SCAN || type == SAF3R_HYBRID; }
+
 // Derived layout numbers.
 struct Dims {
   int S, gh, gw, ns, H, dino_dim;
@@ -73,6 +78,8 @@ struct HeadPlan {
   Seg seg;            // implicit segment
   int32_t radius;     // position heads
   int32_t nb_base;    // position heads: derived row where the cell-major neighbour rows start
+  int32_t lat_stride; // hybrid heads: lattice keys inside a kept tile are counted in the derived run
+  int32_t lat_phase;  //   (so the tile runs mask them); 0 = no lattice mask
 };
 
 struct AttnParams {
@@ -148,7 +155,7 @@ cudaError_t launch_derived(const DerivedArgs& a, bool any_scan, const uint16_t* 
 cudaError_t launch_plan_position(int n_items, int S, int gh, int gw, int ns, int N, int R, int cap, Seg* segs,
                                  int* counts, cudaStream_t stream);
 cudaError_t launch_plan_corr(const int32_t* ranked, const int32_t* order, int kmax, int kt, int T, int N, int V,
-                             int ns, int S, Seg* segs, int cap, int* counts, int* err, cudaStream_t stream);
+                             int ns, int tail_len, Seg* segs, int cap, int* counts, int* err, cudaStream_t stream);
 size_t nmse_workspace_bytes(int H);
 cudaError_t launch_nmse(const float* full, const float* sparse, int H, long long per_head, double* part,
                         double* out, cudaStream_t stream);

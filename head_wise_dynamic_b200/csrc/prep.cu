@@ -47,6 +47,7 @@ __device__ __forceinline__ int derived_token(const DerivedArgs& a, const Derived
       return t;
     }
     case SAF3R_SCAN:
+    case SAF3R_HYBRID:  // the lattice, then the specials off it
       if (r < d.n_lat) return d.phase + r * d.stride;
       return offlists[d.off_list + (r - d.n_lat)];
     default:  // SAF3R_CORR: the special tokens
@@ -78,7 +79,7 @@ __global__ void cache_check_kernel(const CacheHeader* h, uint64_t hash, int N, i
 // Off-lattice special tokens of each scan head, ascending (one warp per head).
 __global__ void scan_specials_kernel(DerivedArgs a, int* offlists) {
   const DerivedHead& d = a.h[blockIdx.x];
-  if (d.kind != SAF3R_SCAN) return;
+  if (!lattice_kind(d.kind)) return;
   const int lane = threadIdx.x;
   const int nsp = a.ns * a.S;
   int base = 0;
@@ -193,7 +194,7 @@ __global__ void plan_position_kernel(int n_items, int S, int gh, int gw, int ns,
 // then the special tokens.  Quarter q of item m is query tile order[4m + q].
 __global__ void __launch_bounds__(256) plan_corr_kernel(const int32_t* __restrict__ ranked,
                                                         const int32_t* __restrict__ order, int kmax, int kt, int T,
-                                                        int N, int V, int ns, int S, Seg* __restrict__ segs,
+                                                        int N, int V, int ns, int tail_len, Seg* __restrict__ segs,
                                                         int cap, int* __restrict__ counts, int* err) {
   extern __shared__ uint32_t memb[];  // [T]
   __shared__ int tmp[32];
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(256) plan_corr_kernel(const int32_t* __restric
   }
   if (threadIdx.x == 0) {
     const int nu = min(base, cap - 1);
-    out[nu] = Seg{1, 0, ns * S, kSegAllQuarters};
+    out[nu] = Seg{1, 0, tail_len, kSegAllQuarters};  // the head's derived rows: specials (and its lattice)
     counts[m] = nu + 1;
   }
 }
@@ -334,7 +335,7 @@ cudaError_t launch_plan_position(int n_items, int S, int gh, int gw, int ns, int
 }
 
 cudaError_t launch_plan_corr(const int32_t* ranked, const int32_t* order, int kmax, int kt, int T, int N, int V,
-                             int ns, int S, Seg* segs, int cap, int* counts, int* err, cudaStream_t stream) {
+                             int ns, int tail_len, Seg* segs, int cap, int* counts, int* err, cudaStream_t stream) {
   const int n_items = (T + 3) / 4;
   const size_t smem = sizeof(uint32_t) * T;
   if (smem > 48 * 1024) {
@@ -342,8 +343,8 @@ cudaError_t launch_plan_corr(const int32_t* ranked, const int32_t* order, int km
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  plan_corr_kernel<<<n_items, 256, smem, stream>>>(ranked, order, kmax, kt, T, N, V, ns, S, segs, cap, counts,
-                                                   err);
+  plan_corr_kernel<<<n_items, 256, smem, stream>>>(ranked, order, kmax, kt, T, N, V, ns, tail_len, segs, cap,
+                                                   counts, err);
   return cudaGetLastError();
 }
 

@@ -54,7 +54,10 @@ typedef enum {
     SAF3R_PROBE = 1,     /* query-probe Top-K: Top-k patch keys by mean-query score, + all specials */
     SAF3R_CORR = 2,      /* DINO Top-K, block-wise: per 64-query tile, Top-k 64-token key tiles + all specials */
     SAF3R_SCAN = 3,      /* uniform sampling: keys j with j mod stride == phase, + all specials */
-    SAF3R_DENSE = 4      /* every key (full attention) */
+    SAF3R_DENSE = 4,     /* every key (full attention) */
+    SAF3R_HYBRID = 5     /* CORR's k key tiles united with SCAN's lattice (stride, phase), + all specials:
+                            the Top-K / uniform-stride combination that section 5.3 ("Further Analysis
+                            of the DINO Top-K kernel") proposes against regions the DINO matches miss */
 } saf3r_head_type;
 
 typedef struct {
@@ -70,9 +73,9 @@ typedef struct {
 
 typedef struct {
     int32_t type;       /* saf3r_head_type */
-    int32_t k;          /* PROBE: kept patch keys (1..S*grid_h*grid_w); CORR: kept key tiles (1..T) */
-    int32_t stride;     /* SCAN: >= 1 */
-    int32_t phase;      /* SCAN: 0 <= phase < stride */
+    int32_t k;          /* PROBE: kept patch keys (1..S*grid_h*grid_w); CORR, HYBRID: kept key tiles (1..T) */
+    int32_t stride;     /* SCAN, HYBRID: >= 1 */
+    int32_t phase;      /* SCAN, HYBRID: 0 <= phase < stride */
     int32_t radius;     /* POSITION: neighbourhood radius in cells, 0..3 (1 = 3x3) */
 } saf3r_head_cfg;
 
@@ -83,8 +86,8 @@ enum { SAF3R_OP_SELECT = 0, SAF3R_OP_SPARSE = 1, SAF3R_OP_DENSE = 2, SAF3R_OP_PR
  * Size in bytes of the index cache that saf3r_select_kv fills for this layout
  * and per-head configuration (cfg: H entries).  The cache holds a header with
  * a hash of (layout, cfg), each probe head's kept patch keys (int32, ascending)
- * and, if any head is CORR, the ranked key-tile list of every query tile
- * (int32 [T][kmax], best first; T = ceil(N/64), kmax = largest CORR k).
+ * and, if any head is CORR or HYBRID, the ranked key-tile list of every query
+ * tile (int32 [T][kmax], best first; T = ceil(N/64), kmax = largest such k).
  * Returns 0 for an invalid layout or cfg.
  */
 size_t saf3r_cache_bytes(const saf3r_layout* layout, const saf3r_head_cfg* cfg);
@@ -111,9 +114,12 @@ size_t saf3r_profile_workspace_bytes(const saf3r_layout* layout, const saf3r_hea
  *   - CORR heads: each flat 64-token tile gets the mean of the L2-normalised
  *     DINO features of its patch tokens; tiles are compared by cosine; every
  *     query tile ranks all tiles (itself included; ties to the lower tile).
- *     Computed once and shared by all CORR heads (prefixes serve smaller k).
- *   - POSITION, SCAN and DENSE heads need no cached state.
- * q, k: bf16 [H][N][d]; dino: fp32 patch features, or NULL when no head is CORR.
+ *     Computed once and shared by all CORR and HYBRID heads (prefixes serve
+ *     smaller k).
+ *   - POSITION, SCAN and DENSE heads need no cached state (a HYBRID head's
+ *     lattice neither).
+ * q, k: bf16 [H][N][d]; dino: fp32 patch features, or NULL when no head is CORR
+ * or HYBRID.
  * workspace: saf3r_workspace_bytes(layout, cfg, SAF3R_OP_SELECT) bytes.
  */
 saf3r_status saf3r_select_kv(const saf3r_layout* layout, const saf3r_head_cfg* cfg,
@@ -208,8 +214,8 @@ saf3r_status saf3r_choose_eq2(int n_inputs, int H, int n_cand, const double* nms
 
 /*
  * Copy one head's cached index list to host memory (synchronizes `stream`):
- * PROBE head -> its k kept patch keys (ascending); CORR head -> the ranked
- * tile list int32 [T][k] truncated to that head's k.  *n receives the number
+ * PROBE head -> its k kept patch keys (ascending); CORR or HYBRID head -> the
+ * ranked tile list int32 [T][k] truncated to that head's k.  *n receives the number
  * of entries; at most `cap` are written.  Other head kinds return
  * SAF3R_ERR_INVALID.
  */

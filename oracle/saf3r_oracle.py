@@ -41,7 +41,7 @@ from typing import Dict, List, Sequence
 
 import numpy as np
 
-POSITION, PROBE, CORR, SCAN, DENSE = 0, 1, 2, 3, 4
+POSITION, PROBE, CORR, SCAN, DENSE, HYBRID = 0, 1, 2, 3, 4, 5
 
 
 # ----------------------------------------------------------------------------
@@ -235,7 +235,7 @@ def select(L, heads, Q, K, dino) -> Selection:
             sc = probe_scores(qbar, K[h])
             sel.probe_scores[h] = sc
             sel.probe_keys[h] = probe_topk(L, sc, hc.k)
-        elif hc.kind == CORR:
+        elif hc.kind in (CORR, HYBRID):
             kt_max = max(kt_max, hc.k)
     if kt_max > 0:
         cos = tile_cosines(dino_tile_means(L, dino))
@@ -254,6 +254,10 @@ def key_set(L, hc, sel: Selection, h: int, i: int) -> np.ndarray:
         return stride_set(L, hc.stride, hc.phase)
     if hc.kind == CORR:
         return corr_set(L, sel.tile_rank[i // L.tile, :hc.k])
+    if hc.kind == HYBRID:
+        # section 5.3 ("Further Analysis of the DINO Top-K kernel"): the DINO tiles combined
+        # with uniform striding, i.e. the union of the two kept sets
+        return np.union1d(corr_set(L, sel.tile_rank[i // L.tile, :hc.k]), stride_set(L, hc.stride, hc.phase))
     if hc.kind == DENSE:
         return np.arange(L.N, dtype=np.int64)
     raise ValueError(hc.kind)
@@ -263,7 +267,7 @@ def _group_key(L, hc, i: int):
     """Rows with equal group keys have equal key sets (used only to batch rows)."""
     if hc.kind in (PROBE, SCAN, DENSE):
         return 0
-    if hc.kind == CORR:
+    if hc.kind in (CORR, HYBRID):
         return i // L.tile
     s, loc = token_parts(L, i)
     return -1 if loc < L.n_special else loc
@@ -355,9 +359,9 @@ def choose_eq2(nmse_tables, pairs_tables, base: int) -> List[int]:
 
 
 def apply_candidate(hc, h: int):
-    """A candidate applied to head h: scan candidates take phase = h mod stride."""
-    if hc.kind == SCAN:
-        return type(hc)(SCAN, k=hc.k, stride=hc.stride, phase=h % hc.stride, radius=hc.radius)
+    """A candidate applied to head h: scan and hybrid candidates take phase = h mod stride."""
+    if hc.kind in (SCAN, HYBRID):
+        return type(hc)(hc.kind, k=hc.k, stride=hc.stride, phase=h % hc.stride, radius=hc.radius)
     return hc
 
 

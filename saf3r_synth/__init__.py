@@ -30,8 +30,8 @@ from typing import List, Optional
 import numpy as np
 
 # head kinds (paper section 3, Observation #2; kernels of section 4.1)
-POSITION, PROBE, CORR, SCAN, DENSE = 0, 1, 2, 3, 4
-KIND_NAMES = {POSITION: "position", PROBE: "probe", CORR: "corr", SCAN: "scan", DENSE: "dense"}
+POSITION, PROBE, CORR, SCAN, DENSE, HYBRID = 0, 1, 2, 3, 4, 5
+KIND_NAMES = {POSITION: "position", PROBE: "probe", CORR: "corr", SCAN: "scan", DENSE: "dense", HYBRID: "hybrid"}
 
 N_SPECIAL = 5      # 1 camera + 4 register tokens per view
 HEAD_DIM = 64
@@ -127,6 +127,12 @@ WORKLOADS = {
                      seed=SEED_BASE + 2000),
     "s200": Workload("s200", Layout(S=200, g=37, H=16), M=4096, delta=97, D=1024,
                      heads=_split16(13740, 215, 20), sample_rows=1024, seed=SEED_BASE + 3000),
+    # the S=100 layer with its correspondence heads as tile Top-64 united with a stride-32 lattice
+    "s100_hybrid": Workload("s100_hybrid", Layout(S=100, g=37, H=16), M=4096, delta=97, D=1024,
+                            heads=_split16(8192, 64, 16)[:8] +
+                            [HeadCfg(HYBRID, k=64, stride=32, phase=h % 32) for h in range(8, 12)] +
+                            _split16(8192, 64, 16)[12:],
+                            calls=4, sample_rows=2048, seed=SEED_BASE + 2000),
     "stack": Workload("stack", Layout(S=64, g=37, H=16), M=4096, delta=97, D=1024,
                       heads=_split16(4096, 32, 10), layers=24, sample_rows=256,
                       seed=SEED_BASE + 4000, candidates=_profile_candidates()),

@@ -90,3 +90,13 @@ def test_choose_eq2_rejects_bad_arguments():
     with pytest.raises(hw.Saf3rError):
         hw.saf3r_choose_eq2(E, W, -1)
     assert hw.baseline_stride(0.85) == 7
+
+
+@pytest.mark.parametrize("field,value", [("k", 0), ("k", 18), ("stride", 0), ("phase", 8), ("phase", -1)])
+def test_bad_hybrid_cfg_sizes_zero(field, value):
+    L, cfg = _tiny()
+    cfg[2].type = hw.HYBRID
+    cfg[2].k, cfg[2].stride, cfg[2].phase = 3, 8, 5
+    assert hw.saf3r_cache_bytes(L, cfg) > 0
+    setattr(cfg[2], field, value)
+    assert hw.saf3r_cache_bytes(L, cfg) == 0

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 import oracle as O
-from saf3r_synth import CORR, POSITION, PROBE, SCAN, HeadCfg, Layout, Scene, Workload, bf16_to_f32, qkv
+from saf3r_synth import CORR, HYBRID, POSITION, PROBE, SCAN, HeadCfg, Layout, Scene, Workload, bf16_to_f32, qkv
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -20,7 +20,8 @@ def test_eq2_search_matches_oracle():
     base_stride = hw.baseline_stride(SIGMA)
     assert base_stride == O.baseline_stride(SIGMA) == 7
     cands = [HeadCfg(SCAN, stride=base_stride), HeadCfg(POSITION), HeadCfg(PROBE, k=64), HeadCfg(PROBE, k=128),
-             HeadCfg(CORR, k=1), HeadCfg(CORR, k=2), HeadCfg(SCAN, stride=8), HeadCfg(SCAN, stride=16)]
+             HeadCfg(CORR, k=1), HeadCfg(CORR, k=2), HeadCfg(SCAN, stride=8), HeadCfg(SCAN, stride=16),
+             HeadCfg(HYBRID, k=1, stride=16)]
     scene = Scene(wl)
     dino_np = scene.dino()
     dino = torch.from_numpy(dino_np).cuda()

@@ -5,8 +5,8 @@ import numpy as np
 import pytest
 
 import oracle as O
-from saf3r_synth import (CORR, DENSE, POSITION, PROBE, SCAN, WORKLOADS, HeadCfg, Layout, Scene, Workload,
-                         bf16_to_f32, qkv, sample_rows)
+from saf3r_synth import (CORR, DENSE, HYBRID, POSITION, PROBE, SCAN, WORKLOADS, HeadCfg, Layout, Scene,
+                         Workload, bf16_to_f32, qkv, sample_rows)
 from parity_util import check_probe, check_tiles, compare_outputs
 
 torch = pytest.importorskip("torch")
@@ -52,9 +52,9 @@ def check_selection(case, heads, att, sel):
         if hc.kind == PROBE:
             keys = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h)
             exact[h] = check_probe(keys, case.L, sel, h, hc.k, f"probe head {h}")
-        elif hc.kind == CORR:
+        elif hc.kind in (CORR, HYBRID):
             ranked = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(case.L.T, hc.k)
-            exact[h] = check_tiles(ranked, sel, hc.k, f"corr head {h}")
+            exact[h] = check_tiles(ranked, sel, hc.k, f"tile head {h}")
     return exact
 
 
@@ -122,6 +122,13 @@ EDGE = {
     # larger than one 128-key block per run; big probe K spanning many blocks
     "multi_block": _custom(6, 16, [HeadCfg(PROBE, k=700), HeadCfg(POSITION), HeadCfg(SCAN, stride=2, phase=1),
                                    HeadCfg(CORR, k=9)]),
+    # tiles united with a stride lattice: ragged layout; a lattice of one key per tile; stride 1
+    # (every key); a plain correspondence head with the same budget sharing the tile lists
+    "hybrid_ragged": _custom(3, 9, [HeadCfg(HYBRID, k=2, stride=5, phase=4), HeadCfg(HYBRID, k=1, stride=64, phase=63),
+                                    HeadCfg(HYBRID, k=3, stride=1, phase=0), HeadCfg(CORR, k=2)]),
+    # several blocks per run, two hybrid heads whose derived runs differ in length
+    "hybrid_multi": _custom(6, 16, [HeadCfg(HYBRID, k=9, stride=7, phase=3), HeadCfg(HYBRID, k=4, stride=16, phase=0),
+                                    HeadCfg(SCAN, stride=7, phase=3), HeadCfg(CORR, k=9)]),
 }
 
 
@@ -163,3 +170,17 @@ def test_s32_selection_and_sampled_rows(s32):
     sel = oracle_select(s32, heads)
     exact = check_selection(s32, heads, att, sel)
     check_rows(s32, heads, sel, out, lambda h: sample_rows(s32.wl, h, 512), exact)
+
+
+def test_s32_hybrid_heads_sampled_rows_and_pairs(s32):
+    """Tile Top-32 united with stride-20 lattices (phase = head mod 20) on the S=32 layer."""
+    hw = _hw()
+    heads = [HeadCfg(HYBRID, k=32, stride=20, phase=h % 20) for h in range(s32.L.H)]
+    att, out = run_gpu(s32, heads, out_fp32=False)
+    sel = oracle_select(s32, heads)
+    exact = check_selection(s32, heads, att, sel)
+    check_rows(s32, heads, sel, out, lambda h: sample_rows(s32.wl, h, 256), exact)
+    pairs = hw.saf3r_kept_pairs(att.layout, att.cfg, att.cache)
+    for h in (0, 7):
+        if exact.get(h, True):
+            assert int(pairs[h]) == O.kept_pairs(s32.L, heads[h], sel, h)

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle as O
-from saf3r_synth import CORR, DENSE, POSITION, PROBE, SCAN, HeadCfg, Layout
+from saf3r_synth import CORR, DENSE, HYBRID, POSITION, PROBE, SCAN, HeadCfg, Layout
 
 RNG = np.random.default_rng(1234)
 
@@ -217,7 +217,7 @@ def test_full_budgets_reduce_to_dense():
     rows = np.arange(L.N)
     dense = O.dense_rows(Q[0], K[0], V[0], rows)
     for hc in [HeadCfg(PROBE, k=L.S * L.P), HeadCfg(SCAN, stride=1, phase=0), HeadCfg(CORR, k=L.T),
-               HeadCfg(DENSE)]:
+               HeadCfg(DENSE), HeadCfg(HYBRID, k=1, stride=1, phase=0), HeadCfg(HYBRID, k=L.T, stride=7, phase=2)]:
         sel = O.select(L, [hc], Q, K, dino)
         out = O.sparse_rows(L, hc, sel, 0, Q[0], K[0], V[0], rows)
         np.testing.assert_allclose(out, dense, rtol=0, atol=1e-12)
@@ -301,3 +301,25 @@ def test_choose_eq2_equals_constrained_argmin():
         E, W = Es.mean(axis=0), Ws.mean(axis=0)
         for h, c in enumerate(got):
             assert W[h, c] <= W[h, base] and E[h, c] <= E[h, base]
+
+
+def test_hybrid_set_counts_and_pieces():
+    """The hybrid set is the tile set united with the stride set: its size by inclusion-exclusion
+    over the tokens of the kept tiles, and each piece alone when the other is empty or full."""
+    L = small_layout(S=3, g=7)   # V = 54, N = 162, three tiles (the last one partial)
+    dino = RNG.standard_normal((L.S * L.P, 8)).astype(np.float32)
+    Q = K = RNG.standard_normal((1, L.N, 64)).astype(np.float32)
+    for k, stride, phase in [(1, 5, 3), (2, 9, 0), (1, 64, 63), (3, 2, 1)]:
+        hc = HeadCfg(HYBRID, k=k, stride=stride, phase=phase)
+        sel = O.select(L, [hc], Q, K, dino)
+        lattice = set(range(phase, L.N, stride))
+        specials = {s * L.V + i for s in range(L.S) for i in range(L.n_special)}
+        for i in (0, 60, L.N - 1):
+            tiles = sel.tile_rank[i // 64, :k]
+            tile_tokens = {t for v in tiles for t in range(64 * int(v), min(L.N, 64 * int(v) + 64))}
+            patch_in_tiles = tile_tokens - specials
+            want = len(lattice | specials) + len(patch_in_tiles - lattice)
+            got = O.key_set(L, hc, sel, 0, i)
+            assert len(got) == want and len(set(got.tolist())) == want
+            assert set(got.tolist()) == lattice | specials | patch_in_tiles
+        assert O.kept_pairs(L, hc, sel, 0) == sum(O.kept_count(L, hc, sel, 0, i) for i in range(L.N))
