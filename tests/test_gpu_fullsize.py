@@ -25,9 +25,9 @@ def _check_layer(wl, att, scene, layer, rows_per_head, sel=None):
             if hc.kind == 1:
                 exact[h] = check_probe(hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h), L, sel, h, hc.k,
                                        f"probe head {h}")
-            elif hc.kind == 2:
+            elif hc.kind in (2, 5):  # correspondence and hybrid heads: ranked tiles
                 ranked = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(L.T, hc.k)
-                exact[h] = check_tiles(ranked, sel, hc.k, f"corr head {h}")
+                exact[h] = check_tiles(ranked, sel, hc.k, f"tile head {h}")
         sel.exact = exact
     att.out.fill_(float("nan"))
     out = att(q, k, v)
@@ -60,3 +60,12 @@ def test_s200_layer():
     scene = Scene(wl)
     att = hw.SparseGlobalAttention(wl.layout, wl.heads)
     _check_layer(wl, att, scene, 0, 1024)
+
+
+def test_s100_hybrid_layer():
+    """The S=100 layer with tile Top-64 united with a stride-32 lattice on the correspondence heads."""
+    import head_wise_dynamic_b200 as hw
+    wl = WORKLOADS["s100_hybrid"]
+    scene = Scene(wl)
+    att = hw.SparseGlobalAttention(wl.layout, wl.heads)
+    _check_layer(wl, att, scene, 0, 512)
