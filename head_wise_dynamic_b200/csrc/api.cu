@@ -127,7 +127,7 @@ saf3r_status check_cfg(const Dims& d, const saf3r_head_cfg* cfg, int H) {
     const saf3r_head_cfg& c = cfg[h];
     switch (c.type) {
       case SAF3R_POSITION:
-        if (c.radius < 0 || c.radius > kMaxRadius) return SAF3R_ERR_INVALID;
+        if (c.radius < -1 || c.radius > kMaxRadius) return SAF3R_ERR_INVALID;
         break;
       case SAF3R_PROBE:
         if (c.k < 1 || c.k > d.S * d.P) return SAF3R_ERR_INVALID;
@@ -697,8 +697,10 @@ static long long pairs_of(const Dims& d, const saf3r_head_cfg& c, const std::vec
       long long tot = nsp * base;  // special-token queries
       for (int r = 0; r < d.gh; ++r)
         for (int col = 0; col < d.gw; ++col) {
-          const long long nb = static_cast<long long>(std::min(r + c.radius, d.gh - 1) - std::max(r - c.radius, 0) + 1) *
-                               (std::min(col + c.radius, d.gw - 1) - std::max(col - c.radius, 0) + 1);
+          const long long nb =
+              c.radius < 0 ? 0
+                           : static_cast<long long>(std::min(r + c.radius, d.gh - 1) - std::max(r - c.radius, 0) + 1) *
+                                 (std::min(col + c.radius, d.gw - 1) - std::max(col - c.radius, 0) + 1);
           tot += d.S * (base + (d.S - 1) * nb);
         }
       return tot;

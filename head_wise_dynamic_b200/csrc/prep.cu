@@ -147,7 +147,7 @@ __global__ void plan_position_kernel(int n_items, int S, int gh, int gw, int ns,
   const int i0 = m * kItemRows;
   const int i1 = min(N, i0 + kItemRows);
   const int nb_base = ns * S + P;
-  if (S > 1 && i0 < P * S) {
+  if (S > 1 && i0 < P * S && R >= 0) {  // R < 0: the anchor frame only, no neighbourhood runs
     const int c_lo = i0 / S, c_hi = (min(i1, P * S) - 1) / S;
     const int r_lo = c_lo / gw, r_hi = c_hi / gw;
     int prev_end = -1;

@@ -76,7 +76,8 @@ typedef struct {
     int32_t k;          /* PROBE: kept patch keys (1..S*grid_h*grid_w); CORR, HYBRID: kept key tiles (1..T) */
     int32_t stride;     /* SCAN, HYBRID: >= 1 */
     int32_t phase;      /* SCAN, HYBRID: 0 <= phase < stride */
-    int32_t radius;     /* POSITION: neighbourhood radius in cells, 0..3 (1 = 3x3) */
+    int32_t radius;     /* POSITION: neighbourhood radius in cells, 0..3 (1 = 3x3); -1 = the anchor frame
+                           only (section 4.1's first static example: all queries attend to view 0) */
 } saf3r_head_cfg;
 
 /* Operations for saf3r_workspace_bytes. */

@@ -77,6 +77,7 @@ def position_set(L, i: int, radius: int = 1) -> np.ndarray:
     Query i keeps every special token, every token of the anchor view 0, and,
     when i is a patch token at grid cell (r, c), the cells (r+dr, c+dc) with
     |dr|, |dc| <= radius of every view (clipped at the grid border, no wrap).
+    radius = -1 keeps the anchor frame (and the specials) only.
     """
     keys = set(special_tokens(L).tolist())
     keys.update(range(0, L.V))

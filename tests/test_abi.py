@@ -46,7 +46,7 @@ def test_bad_layout_sizes_zero(field, value):
 
 
 @pytest.mark.parametrize("h,field,value", [(1, "k", 0), (1, "k", 10 ** 6), (2, "k", 18), (3, "stride", 0),
-                                           (3, "phase", 8), (0, "radius", 4), (0, "type", 9)])
+                                           (3, "phase", 8), (0, "radius", 4), (0, "radius", -2), (0, "type", 9)])
 def test_bad_cfg_sizes_zero(h, field, value):
     L, cfg = _tiny()
     setattr(cfg[h], field, value)

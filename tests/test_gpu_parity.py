@@ -118,7 +118,8 @@ EDGE = {
     "full_budgets": _custom(2, 10, [HeadCfg(PROBE, k=200), HeadCfg(CORR, k=4), HeadCfg(SCAN, stride=1),
                                     HeadCfg(DENSE), HeadCfg(POSITION, radius=0), HeadCfg(POSITION, radius=2)]),
     # many views per item (S = 5 < 256): several cells per work item; a 3-head layout
-    "many_cells": _custom(5, 11, [HeadCfg(POSITION), HeadCfg(SCAN, stride=3, phase=1), HeadCfg(CORR, k=5)]),
+    "many_cells": _custom(5, 11, [HeadCfg(POSITION), HeadCfg(SCAN, stride=3, phase=1), HeadCfg(CORR, k=5),
+                                  HeadCfg(POSITION, radius=-1)]),
     # larger than one 128-key block per run; big probe K spanning many blocks
     "multi_block": _custom(6, 16, [HeadCfg(PROBE, k=700), HeadCfg(POSITION), HeadCfg(SCAN, stride=2, phase=1),
                                    HeadCfg(CORR, k=9)]),

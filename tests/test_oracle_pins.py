@@ -323,3 +323,11 @@ def test_hybrid_set_counts_and_pieces():
             assert len(got) == want and len(set(got.tolist())) == want
             assert set(got.tolist()) == lattice | specials | patch_in_tiles
         assert O.kept_pairs(L, hc, sel, 0) == sum(O.kept_count(L, hc, sel, 0, i) for i in range(L.N))
+
+
+def test_anchor_frame_only_static_set():
+    L = small_layout(S=3, g=4)
+    specials = {s * L.V + i for s in range(L.S) for i in range(L.n_special)}
+    want = specials | set(range(L.V))
+    for i in range(L.N):
+        assert set(O.position_set(L, i, radius=-1).tolist()) == want
