@@ -88,7 +88,7 @@ def workload_desc(wl):
     kinds = []
     for h, hc in enumerate(wl.heads):
         p = {1: f" Top-{hc.k}", 2: f" tile Top-{hc.k}", 3: f" stride {hc.stride}",
-             5: f" tile Top-{hc.k} + stride {hc.stride}"}.get(hc.kind, "")
+             5: f" tile Top-{hc.k} + stride {hc.stride}", 6: f" per-frame Top-{hc.k}"}.get(hc.kind, "")
         kinds.append(f"{h}:{KIND_NAMES[hc.kind]}{p}")
     return (f"{wl.name}: S={L.S} views x ({L.g}x{L.g} patches + {L.n_special} special) = {L.N} tokens, "
             f"H={L.H}, d={L.d}; heads [{', '.join(kinds)}]; one index build + {wl.calls} layer calls "

@@ -24,7 +24,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "saf3r.h")
 # saf3r_status
 OK, ERR_INVALID, ERR_CUDA, ERR_TIMEOUT, ERR_INDEX, ERR_UNSUPPORTED = range(6)
 # saf3r_head_type
-POSITION, PROBE, CORR, SCAN, DENSE, HYBRID = range(6)
+POSITION, PROBE, CORR, SCAN, DENSE, HYBRID, TOKEN = range(7)
 # workspace operations
 OP_SELECT, OP_SPARSE, OP_DENSE, OP_PROFILE = range(4)
 

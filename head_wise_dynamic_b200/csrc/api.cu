@@ -144,6 +144,10 @@ saf3r_status check_cfg(const Dims& d, const saf3r_head_cfg* cfg, int H) {
         break;
       case SAF3R_DENSE:
         break;
+      case SAF3R_TOKEN:
+        if (c.k < 1 || c.k > d.P) return SAF3R_ERR_INVALID;
+        if (d.dino_dim > kTokenMaxDim || token_topk_smem_bytes(d.P, c.k) > 200 * 1024) return SAF3R_ERR_UNSUPPORTED;
+        break;
       default:
         return SAF3R_ERR_INVALID;
     }
@@ -165,7 +169,9 @@ uint64_t cache_hash(const saf3r_layout* L, const saf3r_head_cfg* cfg) {
   uint64_t h = 1469598103934665603ull;
   h = fnv1a(h, L, sizeof(saf3r_layout));
   for (int i = 0; i < L->H; ++i) {
-    const int32_t v[2] = {cfg[i].type, (cfg[i].type == SAF3R_PROBE || tile_kind(cfg[i].type)) ? cfg[i].k : 0};
+    const int32_t v[2] = {cfg[i].type,
+                          (cfg[i].type == SAF3R_PROBE || tile_kind(cfg[i].type) || cfg[i].type == SAF3R_TOKEN) ? cfg[i].k
+                                                                                                       : 0};
     h = fnv1a(h, v, sizeof(v));
   }
   return h;
@@ -177,6 +183,8 @@ struct CacheLayout {
   int corr_off = 0;
   int corr_kmax = 0;
   int order_off = 0;
+  int tok_kmax = 0;        // token-wise heads: widest per-frame budget
+  long long tok_off = 0;   // int32 offset of the per-frame lists [S*P][S][tok_kmax]
   size_t bytes = 0;
 };
 
@@ -190,11 +198,15 @@ CacheLayout cache_layout(const Dims& d, const saf3r_head_cfg* cfg) {
       ints += (cfg[h].k + 63) & ~63;
     }
     if (tile_kind(cfg[h].type)) c.corr_kmax = std::max(c.corr_kmax, cfg[h].k);
+    if (cfg[h].type == SAF3R_TOKEN) c.tok_kmax = std::max(c.tok_kmax, cfg[h].k);
   }
   c.corr_off = static_cast<int>(ints);
   ints += static_cast<size_t>(d.T) * c.corr_kmax;
   c.order_off = static_cast<int>(ints);
   if (c.corr_kmax > 0) ints += static_cast<size_t>(d.T);
+  ints = (ints + 63) & ~size_t(63);
+  c.tok_off = static_cast<long long>(ints);
+  ints += static_cast<size_t>(d.S) * d.P * d.S * c.tok_kmax;
   c.bytes = align256(ints * 4);
   return c;
 }
@@ -409,12 +421,24 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   // attention
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
-  std::vector<int> order(d.H);
-  for (int h = 0; h < d.H; ++h) order[h] = h;
+  // token-wise heads run in their own kernel (no shared key runs); the others in the MMA kernel
+  std::vector<int> order;
+  TokenAttnParams tp;
+  std::memset(&tp, 0, sizeof(tp));
+  for (int h = 0; h < d.H; ++h) {
+    if (cfg[h].type == SAF3R_TOKEN) {
+      tp.heads[tp.n_heads] = h;
+      tp.k[tp.n_heads] = cfg[h].k;
+      ++tp.n_heads;
+    } else {
+      order.push_back(h);
+    }
+  }
   std::stable_sort(order.begin(), order.end(),
                    [&](int a, int b) { return est_keys(d, cfg[a], s, a) > est_keys(d, cfg[b], s, b); });
+  const int n_main = static_cast<int>(order.size());
   int item = 0;
-  for (int i = 0; i < d.H; ++i) {
+  for (int i = 0; i < n_main; ++i) {
     const int h = order[i];
     const saf3r_head_cfg& c = cfg[h];
     HeadPlan& hp = p.heads[i];
@@ -450,7 +474,7 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
       }
     }
   }
-  p.n_heads = d.H;
+  p.n_heads = n_main;
   p.total_items = item;
   p.S = d.S; p.gh = d.gh; p.gw = d.gw; p.ns = d.ns; p.V = d.V; p.N = d.N; p.P = d.P;
   p.out_fp32 = out_is_fp32 ? 1 : 0;
@@ -463,21 +487,39 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   p.ok_flag = ok_flag;
   p.wait_budget = kWaitBudget;
 
-  CUtensorMap tq, tk, tv, tqc, tkc, tvc;
-  if (!make_map_3d(&tq, q, d.N, d.H) || !make_map_3d(&tk, k, d.N, d.H) || !make_map_3d(&tv, v, d.N, d.H))
-    return SAF3R_ERR_CUDA;
-  const void* kc_base = s.kc_rows > 0 ? static_cast<const void*>(kc) : k;
-  const void* vc_base = s.kc_rows > 0 ? static_cast<const void*>(vc) : v;
-  const void* qc_base = s.qc_rows > 0 ? static_cast<const void*>(qc) : q;
-  if (!make_map_2d(&tkc, kc_base, s.kc_rows > 0 ? s.kc_rows : 1) ||
-      !make_map_2d(&tvc, vc_base, s.kc_rows > 0 ? s.kc_rows : 1) ||
-      !make_map_2d(&tqc, qc_base, s.qc_rows > 0 ? s.qc_rows : 1))
-    return SAF3R_ERR_CUDA;
   if (t_ev_start && t_ev_stop && cudaEventRecord(t_ev_start, stream) != cudaSuccess) return SAF3R_ERR_CUDA;
-  st = cuda_status(launch_attention(p, tq, tk, tv, tqc, tkc, tvc, dev.sms, stream));
-  ++launches;
-  if (st == SAF3R_OK && t_ev_start && t_ev_stop && cudaEventRecord(t_ev_stop, stream) != cudaSuccess)
-    return SAF3R_ERR_CUDA;
+  if (n_main > 0) {
+    CUtensorMap tq, tk, tv, tqc, tkc, tvc;
+    if (!make_map_3d(&tq, q, d.N, d.H) || !make_map_3d(&tk, k, d.N, d.H) || !make_map_3d(&tv, v, d.N, d.H))
+      return SAF3R_ERR_CUDA;
+    const void* kc_base = s.kc_rows > 0 ? static_cast<const void*>(kc) : k;
+    const void* vc_base = s.kc_rows > 0 ? static_cast<const void*>(vc) : v;
+    const void* qc_base = s.qc_rows > 0 ? static_cast<const void*>(qc) : q;
+    if (!make_map_2d(&tkc, kc_base, s.kc_rows > 0 ? s.kc_rows : 1) ||
+        !make_map_2d(&tvc, vc_base, s.kc_rows > 0 ? s.kc_rows : 1) ||
+        !make_map_2d(&tqc, qc_base, s.qc_rows > 0 ? s.qc_rows : 1))
+      return SAF3R_ERR_CUDA;
+    st = cuda_status(launch_attention(p, tq, tk, tv, tqc, tkc, tvc, dev.sms, stream));
+    ++launches;
+    if (st != SAF3R_OK) return st;
+  }
+  if (tp.n_heads > 0) {
+    tp.N = d.N; tp.S = d.S; tp.V = d.V; tp.ns = d.ns; tp.P = d.P;
+    tp.tok_kmax = cl.tok_kmax;
+    tp.tok_off = cl.tok_off;
+    tp.q = static_cast<const uint16_t*>(q);
+    tp.k_ = static_cast<const uint16_t*>(k);
+    tp.v = static_cast<const uint16_t*>(v);
+    tp.out = out;
+    tp.out_fp32 = out_is_fp32 ? 1 : 0;
+    tp.cache = cache_i;
+    tp.ok_flag = ok_flag;
+    tp.err = dev.err;
+    st = cuda_status(launch_token_attention(tp, dev.sms, stream));
+    ++launches;
+    if (st != SAF3R_OK) return st;
+  }
+  if (t_ev_start && t_ev_stop && cudaEventRecord(t_ev_stop, stream) != cudaSuccess) return SAF3R_ERR_CUDA;
   t_launches += launches;
   return st;
 }
@@ -520,12 +562,13 @@ size_t saf3r_workspace_bytes(const saf3r_layout* L, const saf3r_head_cfg* cfg, i
   if (check_cfg(d, cfg, L->H) != SAF3R_OK) return 0;
   if (op == SAF3R_OP_SELECT) {
     int n_probe = 0;
-    bool corr = false;
+    bool corr = false, tok = false;
     for (int h = 0; h < d.H; ++h) {
       n_probe += cfg[h].type == SAF3R_PROBE;
       corr |= tile_kind(cfg[h].type);
+      tok |= cfg[h].type == SAF3R_TOKEN;
     }
-    return select_workspace_bytes(n_probe, d.N, d.T, d.dino_dim, corr);
+    return select_workspace_bytes(n_probe, d.N, d.T, d.dino_dim, corr, tok ? static_cast<long long>(d.S) * d.P : 0);
   }
   if (op == SAF3R_OP_SPARSE) return sparse_layout(d, cfg).total;
   return 0;
@@ -539,7 +582,7 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   const Dims d = make_dims(*L);
   if ((st = check_cfg(d, cfg, L->H)) != SAF3R_OK) return st;
   bool corr = false;
-  for (int h = 0; h < d.H; ++h) corr |= tile_kind(cfg[h].type);
+  for (int h = 0; h < d.H; ++h) corr |= tile_kind(cfg[h].type) || cfg[h].type == SAF3R_TOKEN;
   if (!q || !k || !cache || !workspace || !aligned16(q) || !aligned16(k) || !aligned16(cache) ||
       !aligned16(workspace) || (corr && (!dino || !aligned16(dino))))
     return SAF3R_ERR_INVALID;
@@ -560,6 +603,9 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   sp.corr_kmax = cl.corr_kmax;
   sp.corr_off = cl.corr_off;
   sp.order_off = cl.order_off;
+  sp.S = d.S;
+  sp.tok_kmax = cl.tok_kmax;
+  sp.tok_off = cl.tok_off;
   CacheHeader& hd = sp.header;
   std::memset(&hd, 0, sizeof(hd));
   hd.magic = kCacheMagic;
@@ -570,6 +616,8 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   hd.corr_kmax = cl.corr_kmax;
   hd.corr_off = cl.corr_off;
   hd.order_off = cl.order_off;
+  hd.tok_kmax = cl.tok_kmax;
+  hd.tok_off = cl.tok_off;
   for (int h = 0; h < kMaxHeads; ++h) hd.probe_off[h] = h < d.H ? cl.probe_off[h] : -1;
   int launches = 0;
   cudaError_t e = launch_select(sp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), dino,
@@ -637,6 +685,18 @@ saf3r_status saf3r_cache_export(const saf3r_layout* L, const saf3r_head_cfg* cfg
       return SAF3R_ERR_CUDA;
     return SAF3R_OK;
   }
+  if (c.type == SAF3R_TOKEN) {
+    const size_t rows = static_cast<size_t>(d.S) * d.P * d.S;  // (query patch, frame) pairs
+    *n = rows * c.k;
+    if (!host_idx) return SAF3R_OK;
+    std::vector<int32_t> all(rows * cl.tok_kmax);
+    if (cudaMemcpy(all.data(), base + cl.tok_off, all.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return SAF3R_ERR_CUDA;
+    size_t w = 0;
+    for (size_t u = 0; u < rows && w < cap; ++u)
+      for (int r = 0; r < c.k && w < cap; ++r) host_idx[w++] = all[u * cl.tok_kmax + r];
+    return SAF3R_OK;
+  }
   if (tile_kind(c.type)) {
     *n = static_cast<size_t>(d.T) * c.k;
     if (!host_idx) return SAF3R_OK;
@@ -682,6 +742,8 @@ static long long pairs_of(const Dims& d, const saf3r_head_cfg& c, const std::vec
   switch (c.type) {
     case SAF3R_DENSE:
       return N * N;
+    case SAF3R_TOKEN:  // patch queries: k per frame + the specials; special queries: every key
+      return static_cast<long long>(d.S) * d.P * (static_cast<long long>(d.S) * c.k + nsp) + nsp * N;
     case SAF3R_PROBE:
       return N * (c.k + nsp);
     case SAF3R_SCAN: {

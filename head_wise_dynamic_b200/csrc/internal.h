@@ -11,8 +11,9 @@ constexpr int kTile = 64;         // DINO token tile
 constexpr int kMaxHeads = 64;
 constexpr int kItemRows = 256;    // query rows of one attention work item (two 128-row MMA tiles)
 constexpr int kMaxRadius = 3;
+constexpr int kTokenMaxDim = 384;  // DINO width the token-wise selection keeps in registers
 constexpr uint32_t kCacheMagic = 0x52334653u;  // "SF3R"
-constexpr uint32_t kCacheVersion = 1;
+constexpr uint32_t kCacheVersion = 2;
 
 // Heads whose keys include ranked DINO tiles (they share the cached tile lists), and heads
 // whose keys include the stride lattice (they get the lattice as derived rows).
@@ -44,6 +45,8 @@ struct CacheHeader {
   int32_t corr_kmax;        // width of the ranked tile list (0 = none)
   int32_t corr_off;         // int32 offset of the ranked tile list
   int32_t order_off;        // int32 offset of the query-tile grouping order [T] (correspondence heads)
+  int32_t tok_kmax;         // width of the token-wise per-frame lists (0 = none)
+  int64_t tok_off;          // int32 offset of the token-wise lists [S*P][S][tok_kmax]
   int32_t probe_off[kMaxHeads];  // int32 offset of each probe head's key list (-1 = not a probe head)
 };
 static_assert(sizeof(CacheHeader) <= 512, "cache header too large");
@@ -99,6 +102,23 @@ struct AttnParams {
 };
 
 
+// Token-wise correspondence heads (token_attn.cu): every query row has its own kept keys.
+struct TokenAttnParams {
+  int32_t n_heads;
+  int32_t heads[kMaxHeads];   // head index h
+  int32_t k[kMaxHeads];       // kept patch tokens per frame
+  int32_t N, S, V, ns, P, tok_kmax;
+  long long tok_off;          // int32 offset of the per-frame lists in the cache
+  const uint16_t* q;
+  const uint16_t* k_;
+  const uint16_t* v;
+  void* out;
+  int32_t out_fp32;
+  const int32_t* cache;
+  const int* ok_flag;
+  int* err;
+};
+
 // Selection plan (select.cu).
 struct SelectPlan {
   int N, V, ns, P, T, dim;
@@ -109,6 +129,9 @@ struct SelectPlan {
   int corr_kmax;
   int corr_off;
   int order_off;
+  int S;
+  int tok_kmax;             // token-wise heads: widest per-frame budget (0 = none)
+  long long tok_off;
   CacheHeader header;
 };
 
@@ -144,7 +167,8 @@ size_t attn_smem_bytes();
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmQC, const CUtensorMap& tmKC,
                              const CUtensorMap& tmVC, int num_sms, cudaStream_t stream);
-size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr);
+size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows);
+size_t token_topk_smem_bytes(int P, int kmax);
 cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_t* k, const float* dino,
                           int32_t* cache, uint8_t* ws, cudaStream_t stream, int* n_launch);
 cudaError_t launch_cache_check(const void* cache, uint64_t hash, int N, int T, int* ok, int* err,
@@ -156,6 +180,7 @@ cudaError_t launch_plan_position(int n_items, int S, int gh, int gw, int ns, int
                                  int* counts, cudaStream_t stream);
 cudaError_t launch_plan_corr(const int32_t* ranked, const int32_t* order, int kmax, int kt, int T, int N, int V,
                              int ns, int tail_len, Seg* segs, int cap, int* counts, int* err, cudaStream_t stream);
+cudaError_t launch_token_attention(const TokenAttnParams& p, int num_sms, cudaStream_t stream);
 size_t nmse_workspace_bytes(int H);
 cudaError_t launch_nmse(const float* full, const float* sparse, int H, long long per_head, double* part,
                         double* out, cudaStream_t stream);

@@ -379,30 +379,29 @@ constexpr float kTkBand = 4e-6f;
 
 __device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
-__global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __restrict__ tilevec, int T, int dim,
-                                                             int kmax, int32_t* __restrict__ ranked) {
-  extern __shared__ uint8_t tk_smem[];
-  float* cs = reinterpret_cast<float*>(tk_smem);                               // [8][T]
-  int* hist = reinterpret_cast<int*>(cs + static_cast<size_t>(kTkRows) * T);  // [8 warps][256]
-  int* sel_idx = hist + 8 * 256;                                               // [8 warps][kmax]
-  uint32_t* sel_key = reinterpret_cast<uint32_t*>(sel_idx + 8 * kmax);         // [8 warps][kmax]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u0 = blockIdx.x * kTkRows;
-  const int nr = min(kTkRows, T - u0);
-
-  float4 q[kTkRows][kTkChunks];
+// This lane's slice of kTkRows unit vectors (rows u0.. of `vec`; absent rows and features are 0).
+__device__ __forceinline__ void load_row_slices(const float* __restrict__ vec, int u0, int nr, int dim, int lane,
+                                                float4 (&q)[kTkRows][kTkChunks]) {
 #pragma unroll
   for (int r = 0; r < kTkRows; ++r)
 #pragma unroll
     for (int c = 0; c < kTkChunks; ++c) {
       const int d = 128 * c + 4 * lane;
-      q[r][c] = (r < nr && d < dim) ? ld_f4(tilevec + static_cast<size_t>(u0 + r) * dim + d)
+      q[r][c] = (r < nr && d < dim) ? ld_f4(vec + static_cast<size_t>(u0 + r) * dim + d)
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+}
+
+// fp32 dots of the kTkRows query vectors with candidates cand[0..n) (unit vectors, row-major,
+// `dim` wide) into cs[r * ld + v]: each warp takes one candidate at a time with coalesced loads
+// and folds its eight partial dots over the warp with a transposing butterfly (after it, lane
+// group (lane>>2)&7 holds row r's full dot).  All warps of the block take part.
+__device__ __forceinline__ void dots_fp32(const float4 (&q)[kTkRows][kTkChunks], const float* __restrict__ cand,
+                                          int n, int dim, int nr, float* cs, int ld, int warp, int lane) {
   const int b2 = (lane >> 2) & 1, b3 = (lane >> 3) & 1, b4 = (lane >> 4) & 1;
   const int my_row = (lane >> 2) & 7;
-  for (int v = warp; v < T; v += 8) {
-    const float* fv = tilevec + static_cast<size_t>(v) * dim;
+  for (int v = warp; v < n; v += 8) {
+    const float* fv = cand + static_cast<size_t>(v) * dim;
     float a[kTkRows];
 #pragma unroll
     for (int r = 0; r < kTkRows; ++r) a[r] = 0.f;
@@ -420,7 +419,6 @@ __global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __rest
         }
       }
     }
-    // transposing butterfly: 8 values per lane -> lane group g = (lane>>2)&7 holds row g's sum
     float h4[4], h2[2];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -439,26 +437,28 @@ __global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __rest
     }
     h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
     h1 += __shfl_xor_sync(0xffffffffu, h1, 1);
-    if ((lane & 3) == 0 && my_row < nr) cs[static_cast<size_t>(my_row) * T + v] = h1;
+    if ((lane & 3) == 0 && my_row < nr) cs[static_cast<size_t>(my_row) * ld + v] = h1;
   }
-  __syncthreads();
-  if (warp >= nr) return;
-  float* row = cs + static_cast<size_t>(warp) * T;
-  int* wh = hist + warp * 256;
+}
+
+// One warp: rank row[0..n) (fp32 dots of query row `rq` with candidates cand[0..n)) exactly.
+// Every candidate within kTkBand of the fp32 kmax-th value gets its exact value (fp64 dot,
+// rounded to fp32), then the row is ranked; out[0..kmax) receives candidate indices.
+__device__ __forceinline__ void rank_row_exact(float* row, int n, int kmax, const float4 (&q)[kTkRows][kTkChunks],
+                                               int rq, const float* __restrict__ cand, int dim, int* wh, int* widx,
+                                               uint32_t* wkey, int lane, int32_t* __restrict__ out) {
   uint32_t prefix;
   int remaining;
-  warp_radix_kth(row, T, kmax, wh, lane, prefix, remaining);
+  warp_radix_kth(row, n, kmax, wh, lane, prefix, remaining);
   const float thr = key_value(prefix) - kTkBand;
-  // exact values for every tile within the band: fp64 dot of this warp's query tile (the
-  // registers of row `warp`) with tile v, rounded to fp32
-  for (int v0 = 0; v0 < T; v0 += 32) {
+  for (int v0 = 0; v0 < n; v0 += 32) {
     const int v = v0 + lane;
-    uint32_t todo = __ballot_sync(0xffffffffu, v < T && row[v] >= thr);
+    uint32_t todo = __ballot_sync(0xffffffffu, v < n && row[v] >= thr);
     while (todo) {
       const int bit = __ffs(todo) - 1;
       todo &= todo - 1;
       const int w = v0 + bit;
-      const float* fv = tilevec + static_cast<size_t>(w) * dim;
+      const float* fv = cand + static_cast<size_t>(w) * dim;
       double acc = 0.0;
 #pragma unroll
       for (int c = 0; c < kTkChunks; ++c) {
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __rest
           float4 qa = q[0][c];
 #pragma unroll
           for (int r = 1; r < kTkRows; ++r)
-            if (r == warp) qa = q[r][c];
+            if (r == rq) qa = q[r][c];
           acc = fma(static_cast<double>(qa.x), static_cast<double>(b.x), acc);
           acc = fma(static_cast<double>(qa.y), static_cast<double>(b.y), acc);
           acc = fma(static_cast<double>(qa.z), static_cast<double>(b.z), acc);
@@ -481,8 +481,71 @@ __global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __rest
     }
   }
   __syncwarp();
-  warp_rank_row(row, T, kmax, wh, sel_idx + warp * kmax, sel_key + warp * kmax, lane,
-                ranked + static_cast<size_t>(u0 + warp) * kmax);
+  warp_rank_row(row, n, kmax, wh, widx, wkey, lane, out);
+}
+
+__global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __restrict__ tilevec, int T, int dim,
+                                                             int kmax, int32_t* __restrict__ ranked) {
+  extern __shared__ uint8_t tk_smem[];
+  float* cs = reinterpret_cast<float*>(tk_smem);                               // [8][T]
+  int* hist = reinterpret_cast<int*>(cs + static_cast<size_t>(kTkRows) * T);  // [8 warps][256]
+  int* sel_idx = hist + 8 * 256;                                               // [8 warps][kmax]
+  uint32_t* sel_key = reinterpret_cast<uint32_t*>(sel_idx + 8 * kmax);         // [8 warps][kmax]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u0 = blockIdx.x * kTkRows;
+  const int nr = min(kTkRows, T - u0);
+  float4 q[kTkRows][kTkChunks];
+  load_row_slices(tilevec, u0, nr, dim, lane, q);
+  dots_fp32(q, tilevec, T, dim, nr, cs, T, warp, lane);
+  __syncthreads();
+  if (warp >= nr) return;
+  rank_row_exact(cs + static_cast<size_t>(warp) * T, T, kmax, q, warp, tilevec, dim, hist + warp * 256,
+                 sel_idx + warp * kmax, sel_key + warp * kmax, lane, ranked + static_cast<size_t>(u0 + warp) * kmax);
+}
+
+// ---- token-wise DINO Top-K (section 4.1, "DINO Top-K Kernel": per query token, the Top-K most
+// similar tokens of every frame; section 5.1: K per frame)
+
+// Unit DINO features, one warp per patch token: fp64 sum of squares, one scale in fp32.
+__global__ void __launch_bounds__(256) unit_features_kernel(const float* __restrict__ dino, int rows, int dim,
+                                                            float* __restrict__ unit) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const float* f = dino + static_cast<size_t>(warp) * dim;
+  double ss = 0.0;
+  for (int c = lane; c < dim; c += 32) ss += static_cast<double>(f[c]) * f[c];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = ss > 0.0 ? static_cast<float>(1.0 / sqrt(ss)) : 0.f;
+  for (int c = lane; c < dim; c += 32) unit[static_cast<size_t>(warp) * dim + c] = f[c] * inv;
+}
+
+// Eight query patch tokens per block; for every frame s the fp32 cosines against the frame's P
+// patch tokens, then each warp ranks its query's frame exactly (as the tile form) and writes
+// the kmax best patch indices to lists[(a * S + s) * kmax + rank], a = query's feature row.
+__global__ void __launch_bounds__(256) token_topk_kernel(const float* __restrict__ unit, int S, int P, int dim,
+                                                         int kmax, int32_t* __restrict__ lists) {
+  extern __shared__ uint8_t tk_smem[];
+  float* cs = reinterpret_cast<float*>(tk_smem);                               // [8][P]
+  int* hist = reinterpret_cast<int*>(cs + static_cast<size_t>(kTkRows) * P);  // [8 warps][256]
+  int* sel_idx = hist + 8 * 256;                                               // [8 warps][kmax]
+  uint32_t* sel_key = reinterpret_cast<uint32_t*>(sel_idx + 8 * kmax);         // [8 warps][kmax]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows = S * P;
+  const int a0 = blockIdx.x * kTkRows;
+  const int nr = min(kTkRows, rows - a0);
+  float4 q[kTkRows][kTkChunks];
+  load_row_slices(unit, a0, nr, dim, lane, q);
+  for (int s = 0; s < S; ++s) {
+    const float* cand = unit + static_cast<size_t>(s) * P * dim;
+    dots_fp32(q, cand, P, dim, nr, cs, P, warp, lane);
+    __syncthreads();
+    if (warp < nr)
+      rank_row_exact(cs + static_cast<size_t>(warp) * P, P, kmax, q, warp, cand, dim, hist + warp * 256,
+                     sel_idx + warp * kmax, sel_key + warp * kmax, lane,
+                     lists + (static_cast<size_t>(a0 + warp) * S + s) * kmax);
+    __syncthreads();
+  }
 }
 
 // ---- query-tile grouping of the correspondence heads (a scheduling aid, cached with the indices)
@@ -609,7 +672,7 @@ __global__ void cache_header_kernel(CacheHeader h, CacheHeader* dst) {
 
 }  // namespace
 
-size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr) {
+size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows) {
   size_t b = 0;
   b += static_cast<size_t>(n_probe) * kProbePartials * kD * sizeof(double);
   b += static_cast<size_t>(n_probe) * kD * sizeof(float);
@@ -623,7 +686,13 @@ size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr) {
     b = (b + 255) & ~size_t(255);
     b += static_cast<size_t>(T) * sizeof(int32_t);                      // sorted tiles
   }
-  return b + 256;
+  b = ((b + 255) & ~size_t(255)) + 256;
+  b += static_cast<size_t>(tok_rows) * dim * sizeof(float);  // unit features of the token-wise heads
+  return b;
+}
+
+size_t token_topk_smem_bytes(int P, int kmax) {
+  return sizeof(float) * static_cast<size_t>(kTkRows) * P + sizeof(int) * (8 * 256 + 16 * static_cast<size_t>(kmax));
 }
 
 
@@ -717,6 +786,20 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
       identity_order_kernel<<<(sp.T + 255) / 256, 256, 0, stream>>>(sp.T, order);
       *n_launch += 1;
     }
+  }
+  if (sp.tok_kmax > 0) {
+    // unit features after everything else of the workspace
+    float* unit = reinterpret_cast<float*>(ws + select_workspace_bytes(sp.n_probe, sp.N, sp.T, sp.dim,
+                                                                        sp.corr_kmax > 0, 0));
+    const int rows = sp.S * sp.P;
+    unit_features_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(dino, rows, sp.dim, unit);
+    const size_t smem = token_topk_smem_bytes(sp.P, sp.tok_kmax);
+    cudaError_t e =
+        cudaFuncSetAttribute(token_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    token_topk_kernel<<<(rows + kTkRows - 1) / kTkRows, 256, smem, stream>>>(unit, sp.S, sp.P, sp.dim, sp.tok_kmax,
+                                                                             cache + sp.tok_off);
+    *n_launch += 2;
   }
   return cudaGetLastError();
 }

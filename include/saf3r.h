@@ -55,9 +55,12 @@ typedef enum {
     SAF3R_CORR = 2,      /* DINO Top-K, block-wise: per 64-query tile, Top-k 64-token key tiles + all specials */
     SAF3R_SCAN = 3,      /* uniform sampling: keys j with j mod stride == phase, + all specials */
     SAF3R_DENSE = 4,     /* every key (full attention) */
-    SAF3R_HYBRID = 5     /* CORR's k key tiles united with SCAN's lattice (stride, phase), + all specials:
+    SAF3R_HYBRID = 5,    /* CORR's k key tiles united with SCAN's lattice (stride, phase), + all specials:
                             the Top-K / uniform-stride combination that section 5.3 ("Further Analysis
                             of the DINO Top-K kernel") proposes against regions the DINO matches miss */
+    SAF3R_TOKEN = 6      /* DINO Top-K, token-wise: a patch query keeps, in every frame, the k patch tokens of
+                            highest DINO cosine (section 4.1; section 5.1 sets k per frame), + all specials;
+                            a special-token query (no DINO feature) keeps every key */
 } saf3r_head_type;
 
 typedef struct {
@@ -73,7 +76,8 @@ typedef struct {
 
 typedef struct {
     int32_t type;       /* saf3r_head_type */
-    int32_t k;          /* PROBE: kept patch keys (1..S*grid_h*grid_w); CORR, HYBRID: kept key tiles (1..T) */
+    int32_t k;          /* PROBE: kept patch keys (1..S*grid_h*grid_w); CORR, HYBRID: kept key tiles (1..T);
+                           TOKEN: kept patch tokens per frame (1..grid_h*grid_w) */
     int32_t stride;     /* SCAN, HYBRID: >= 1 */
     int32_t phase;      /* SCAN, HYBRID: 0 <= phase < stride */
     int32_t radius;     /* POSITION: neighbourhood radius in cells, 0..3 (1 = 3x3); -1 = the anchor frame
@@ -88,7 +92,9 @@ enum { SAF3R_OP_SELECT = 0, SAF3R_OP_SPARSE = 1, SAF3R_OP_DENSE = 2, SAF3R_OP_PR
  * and per-head configuration (cfg: H entries).  The cache holds a header with
  * a hash of (layout, cfg), each probe head's kept patch keys (int32, ascending)
  * and, if any head is CORR or HYBRID, the ranked key-tile list of every query
- * tile (int32 [T][kmax], best first; T = ceil(N/64), kmax = largest such k).
+ * tile (int32 [T][kmax], best first; T = ceil(N/64), kmax = largest such k),
+ * and, if any head is TOKEN, the ranked per-frame lists of every patch query
+ * (int32 [S*P][S][kmax] patch indices, best first; kmax = largest TOKEN k).
  * Returns 0 for an invalid layout or cfg.
  */
 size_t saf3r_cache_bytes(const saf3r_layout* layout, const saf3r_head_cfg* cfg);
@@ -117,10 +123,17 @@ size_t saf3r_profile_workspace_bytes(const saf3r_layout* layout, const saf3r_hea
  *     query tile ranks all tiles (itself included; ties to the lower tile).
  *     Computed once and shared by all CORR and HYBRID heads (prefixes serve
  *     smaller k).
+ *   - TOKEN heads: L2-normalised DINO features; for every patch query and
+ *     every frame, the frame's patch tokens ranked by cosine (own token
+ *     included; ties to the lower patch index); the lists are cached.
+ *     The cosines are formed in fp32 and every candidate within the fp32
+ *     error bound of the k-th value is recomputed exactly (fp64), so the
+ *     ranking is that of the fp64 cosines rounded to fp32.  Needs
+ *     dino_dim <= 384 (SAF3R_ERR_UNSUPPORTED otherwise).
  *   - POSITION, SCAN and DENSE heads need no cached state (a HYBRID head's
  *     lattice neither).
- * q, k: bf16 [H][N][d]; dino: fp32 patch features, or NULL when no head is CORR
- * or HYBRID.
+ * q, k: bf16 [H][N][d]; dino: fp32 patch features, or NULL when no head is
+ * CORR, HYBRID or TOKEN.
  * workspace: saf3r_workspace_bytes(layout, cfg, SAF3R_OP_SELECT) bytes.
  */
 saf3r_status saf3r_select_kv(const saf3r_layout* layout, const saf3r_head_cfg* cfg,
@@ -216,7 +229,8 @@ saf3r_status saf3r_choose_eq2(int n_inputs, int H, int n_cand, const double* nms
 /*
  * Copy one head's cached index list to host memory (synchronizes `stream`):
  * PROBE head -> its k kept patch keys (ascending); CORR or HYBRID head -> the
- * ranked tile list int32 [T][k] truncated to that head's k.  *n receives the number
+ * ranked tile list int32 [T][k] truncated to that head's k; TOKEN head -> the
+ * per-frame lists int32 [S*P][S][k] (patch indices) truncated to its k.  *n receives the number
  * of entries; at most `cap` are written.  Other head kinds return
  * SAF3R_ERR_INVALID.
  */

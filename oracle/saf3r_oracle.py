@@ -41,7 +41,7 @@ from typing import Dict, List, Sequence
 
 import numpy as np
 
-POSITION, PROBE, CORR, SCAN, DENSE, HYBRID = 0, 1, 2, 3, 4, 5
+POSITION, PROBE, CORR, SCAN, DENSE, HYBRID, TOKEN = 0, 1, 2, 3, 4, 5, 6
 
 
 # ----------------------------------------------------------------------------
@@ -184,6 +184,37 @@ def corr_set(L, tiles: Sequence[int]) -> np.ndarray:
     return np.unique(np.concatenate(parts))
 
 
+def unit_features(dino: np.ndarray) -> np.ndarray:
+    """L2-normalised DINO features of the patch tokens, fp64 [S*P][dim]."""
+    f = np.asarray(dino, dtype=np.float64)
+    return f / np.linalg.norm(f, axis=1, keepdims=True)
+
+
+def token_topk_row(L, unit: np.ndarray, i: int, k: int) -> np.ndarray:
+    """Token-wise DINO Top-K (section 4.1, "DINO Top-K Kernel"; section 5.1: K per frame): for the
+    patch query token i, in every frame s the k patch tokens of highest cosine (fp64 dot of unit
+    features, rounded to fp32; its own token included; ties to the lower patch index), in rank
+    order, as patch indices.  int64 [S][k]."""
+    s_i, loc = token_parts(L, int(i))
+    a = s_i * L.P + (loc - L.n_special)
+    cos32 = (unit @ unit[a]).astype(np.float32)
+    out = np.empty((L.S, k), dtype=np.int64)
+    for sv in range(L.S):
+        out[sv] = topk_desc(cos32[sv * L.P:(sv + 1) * L.P], k)
+    return out
+
+
+def token_set(L, unit: np.ndarray, i: int, k: int) -> np.ndarray:
+    """Key set of a token-wise correspondence head for query i: the per-frame Top-K patch tokens
+    plus every special token; a special-token query (no DINO feature) keeps every key."""
+    s_i, loc = token_parts(L, int(i))
+    if loc < L.n_special:
+        return np.arange(L.N, dtype=np.int64)
+    p = token_topk_row(L, unit, i, k)
+    toks = (np.arange(L.S, dtype=np.int64)[:, None] * L.V + L.n_special + p).ravel()
+    return np.union1d(toks, special_tokens(L)).astype(np.int64)
+
+
 # ----------------------------------------------------------------------------
 # attention (section 4.1: exact softmax over the kept keys)
 # ----------------------------------------------------------------------------
@@ -223,6 +254,7 @@ class Selection:
         self.probe_keys: Dict[int, np.ndarray] = {}
         self.probe_scores: Dict[int, np.ndarray] = {}
         self.tile_rank: np.ndarray | None = None
+        self.unit: np.ndarray | None = None  # unit DINO features (token-wise heads; their sets are computed per row)
         self.tile_cos: np.ndarray | None = None
 
 
@@ -238,6 +270,8 @@ def select(L, heads, Q, K, dino) -> Selection:
             sel.probe_keys[h] = probe_topk(L, sc, hc.k)
         elif hc.kind in (CORR, HYBRID):
             kt_max = max(kt_max, hc.k)
+        elif hc.kind == TOKEN and sel.unit is None:
+            sel.unit = unit_features(dino)
     if kt_max > 0:
         cos = tile_cosines(dino_tile_means(L, dino))
         sel.tile_cos = cos
@@ -259,6 +293,8 @@ def key_set(L, hc, sel: Selection, h: int, i: int) -> np.ndarray:
         # section 5.3 ("Further Analysis of the DINO Top-K kernel"): the DINO tiles combined
         # with uniform striding, i.e. the union of the two kept sets
         return np.union1d(corr_set(L, sel.tile_rank[i // L.tile, :hc.k]), stride_set(L, hc.stride, hc.phase))
+    if hc.kind == TOKEN:
+        return token_set(L, sel.unit, i, hc.k)
     if hc.kind == DENSE:
         return np.arange(L.N, dtype=np.int64)
     raise ValueError(hc.kind)
@@ -270,6 +306,9 @@ def _group_key(L, hc, i: int):
         return 0
     if hc.kind in (CORR, HYBRID):
         return i // L.tile
+    if hc.kind == TOKEN:  # every patch query has its own set; special queries keep every key
+        s, loc = token_parts(L, i)
+        return -1 if loc < L.n_special else i
     s, loc = token_parts(L, i)
     return -1 if loc < L.n_special else loc
 
@@ -293,6 +332,11 @@ def kept_count(L, hc, sel: Selection, h: int, i: int) -> int:
 
 def kept_pairs(L, hc, sel: Selection, h: int) -> int:
     """Exact number of (query, kept key) pairs of a head over all N queries."""
+    if hc.kind == TOKEN:
+        # per patch query S*k patch keys (distinct frames are disjoint) + the specials; special
+        # queries every key (the per-row sets agree with this count: tests/test_oracle_pins.py)
+        nsp = L.S * L.n_special
+        return L.S * L.P * (L.S * hc.k + nsp) + nsp * L.N
     total = 0
     seen: Dict[object, int] = {}
     for i in range(L.N):

@@ -30,8 +30,9 @@ from typing import List, Optional
 import numpy as np
 
 # head kinds (paper section 3, Observation #2; kernels of section 4.1)
-POSITION, PROBE, CORR, SCAN, DENSE, HYBRID = 0, 1, 2, 3, 4, 5
-KIND_NAMES = {POSITION: "position", PROBE: "probe", CORR: "corr", SCAN: "scan", DENSE: "dense", HYBRID: "hybrid"}
+POSITION, PROBE, CORR, SCAN, DENSE, HYBRID, TOKEN = 0, 1, 2, 3, 4, 5, 6
+KIND_NAMES = {POSITION: "position", PROBE: "probe", CORR: "corr", SCAN: "scan", DENSE: "dense", HYBRID: "hybrid",
+              TOKEN: "token"}
 
 N_SPECIAL = 5      # 1 camera + 4 register tokens per view
 HEAD_DIM = 64
@@ -127,6 +128,10 @@ WORKLOADS = {
                      seed=SEED_BASE + 2000),
     "s200": Workload("s200", Layout(S=200, g=37, H=16), M=4096, delta=97, D=1024,
                      heads=_split16(13740, 215, 20), sample_rows=1024, seed=SEED_BASE + 3000),
+    # the S=32 layer with its position heads replaced by token-wise per-frame DINO Top-16 heads
+    "s32_token": Workload("s32_token", Layout(S=32, g=37, H=16), M=4096, delta=97, D=1024,
+                          heads=[HeadCfg(TOKEN, k=16)] * 4 + _split16(4096, 32, 10)[4:],
+                          sample_rows=256, seed=SEED_BASE + 1000),
     # the S=100 layer with its correspondence heads as tile Top-64 united with a stride-32 lattice
     "s100_hybrid": Workload("s100_hybrid", Layout(S=100, g=37, H=16), M=4096, delta=97, D=1024,
                             heads=_split16(8192, 64, 16)[:8] +

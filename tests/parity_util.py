@@ -51,3 +51,21 @@ def check_tiles(gpu_ranked, sel, k, what):
         ranked = O.topk_desc(sel.tile_cos[u], min(T, k + 8))
         exact &= check_topk_set(gpu_ranked[u], ranked, sel.tile_cos[u], k, f"{what} tile {u}")
     return exact
+
+
+def check_token_lists(gpu_lists, L, unit, k, rows, what):
+    """gpu_lists: int [S*P][S][k] per-frame patch lists of the token-wise head; rows: query
+    tokens (patch tokens are checked, special ones have no list).  Each (row, frame) set must
+    equal the oracle's Top-k up to the boundary band.  Returns True when all are identical."""
+    exact = True
+    for i in rows:
+        s_i, loc = O.token_parts(L, int(i))
+        if loc < L.n_special:
+            continue
+        a = s_i * L.P + loc - L.n_special
+        cos32 = (unit @ unit[a]).astype(np.float32)
+        for sv in range(L.S):
+            frame = cos32[sv * L.P:(sv + 1) * L.P]
+            ranked = O.topk_desc(frame, min(L.P, k + 8))
+            exact &= check_topk_set(gpu_lists[a, sv], ranked, frame, k, f"{what} row {int(i)} frame {sv}")
+    return exact

@@ -100,3 +100,16 @@ def test_bad_hybrid_cfg_sizes_zero(field, value):
     assert hw.saf3r_cache_bytes(L, cfg) > 0
     setattr(cfg[2], field, value)
     assert hw.saf3r_cache_bytes(L, cfg) == 0
+
+
+def test_token_cfg_validation():
+    L, cfg = _tiny()
+    cfg[2].type = hw.TOKEN
+    cfg[2].k = 16
+    assert hw.saf3r_cache_bytes(L, cfg) > 0
+    for k in (0, L.grid_h * L.grid_w + 1):
+        cfg[2].k = k
+        assert hw.saf3r_cache_bytes(L, cfg) == 0
+    cfg[2].k = 4
+    L.dino_dim = 388  # beyond what the token-wise selection keeps in registers: unsupported
+    assert hw.saf3r_cache_bytes(L, cfg) == 0

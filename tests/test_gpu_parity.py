@@ -5,9 +5,9 @@ import numpy as np
 import pytest
 
 import oracle as O
-from saf3r_synth import (CORR, DENSE, HYBRID, POSITION, PROBE, SCAN, WORKLOADS, HeadCfg, Layout, Scene,
+from saf3r_synth import (CORR, DENSE, HYBRID, POSITION, PROBE, SCAN, TOKEN, WORKLOADS, HeadCfg, Layout, Scene,
                          Workload, bf16_to_f32, qkv, sample_rows)
-from parity_util import check_probe, check_tiles, compare_outputs
+from parity_util import check_probe, check_tiles, check_token_lists, compare_outputs
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -185,3 +185,58 @@ def test_s32_hybrid_heads_sampled_rows_and_pairs(s32):
     for h in (0, 7):
         if exact.get(h, True):
             assert int(pairs[h]) == O.kept_pairs(s32.L, heads[h], sel, h)
+
+
+# ---------------------------------------------------------------- token-wise per-frame DINO Top-K
+
+TOKEN_CASES = {
+    # ragged layout; k = P keeps every key; k = 1; a main-kernel head beside them
+    "token_ragged": _custom(3, 9, [HeadCfg(TOKEN, k=3), HeadCfg(TOKEN, k=81), HeadCfg(TOKEN, k=1),
+                                   HeadCfg(SCAN, stride=5, phase=4)]),
+    # token-wise heads mixed with the other kinds in one call
+    "token_mixed": _custom(4, 16, [HeadCfg(TOKEN, k=16), HeadCfg(CORR, k=4), HeadCfg(TOKEN, k=5),
+                                   HeadCfg(POSITION)], D=256),
+}
+
+
+def _check_token_heads(case, heads, att, sel, rows):
+    hw = _hw()
+    L = case.L
+    exact = {}
+    for h, hc in enumerate(heads):
+        if hc.kind != TOKEN:
+            continue
+        lists = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(L.S * L.P, L.S, hc.k)
+        exact[h] = check_token_lists(lists, L, sel.unit, hc.k, rows, f"token head {h}")
+    return exact
+
+
+@pytest.mark.parametrize("name", list(TOKEN_CASES))
+def test_token_heads_all_rows(name):
+    hw = _hw()
+    case = Case(TOKEN_CASES[name])
+    heads = case.wl.heads
+    att, out = run_gpu(case, heads)
+    sel = oracle_select(case, heads)
+    exact = check_selection(case, heads, att, sel)
+    exact.update(_check_token_heads(case, heads, att, sel, np.arange(case.L.N)))
+    check_rows(case, heads, sel, out, lambda h: np.arange(case.L.N), exact)
+    pairs = hw.saf3r_kept_pairs(att.layout, att.cfg, att.cache)
+    for h, hc in enumerate(heads):
+        if hc.kind == TOKEN:
+            assert int(pairs[h]) == sum(O.kept_count(case.L, hc, sel, h, i) for i in range(case.L.N))
+
+
+def test_s32_token_heads_sampled_rows(s32):
+    """Per-frame Top-16 token-wise heads on the S=32 layer (the other heads as configured)."""
+    heads = [HeadCfg(TOKEN, k=16)] * 4 + list(s32.wl.heads[4:])
+    att, out = run_gpu(s32, heads, out_fp32=False)
+    sel = oracle_select(s32, heads)
+    exact = check_selection(s32, heads, att, sel)
+    rows = {h: sample_rows(s32.wl, h, 64) for h in range(4)}
+    hw = _hw()
+    L = s32.L
+    for h in range(4):
+        lists = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(L.S * L.P, L.S, 16)
+        exact[h] = check_token_lists(lists, L, sel.unit, 16, rows[h], f"token head {h}")
+    check_rows(s32, heads, sel, out, lambda h: rows[h] if h < 4 else sample_rows(s32.wl, h, 128), exact)

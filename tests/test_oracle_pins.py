@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle as O
-from saf3r_synth import CORR, DENSE, HYBRID, POSITION, PROBE, SCAN, HeadCfg, Layout
+from saf3r_synth import CORR, DENSE, HYBRID, POSITION, PROBE, SCAN, TOKEN, HeadCfg, Layout
 
 RNG = np.random.default_rng(1234)
 
@@ -331,3 +331,31 @@ def test_anchor_frame_only_static_set():
     want = specials | set(range(L.V))
     for i in range(L.N):
         assert set(O.position_set(L, i, radius=-1).tolist()) == want
+
+
+def test_token_topk_brute_force_and_counts():
+    """Token-wise per-frame Top-K against a brute-force sort of explicit cosines, the own token
+    first in its own frame, k = P reducing to every key, and the closed-form pair count."""
+    L = small_layout(S=3, g=4)   # P = 16 patches per frame
+    dino = RNG.standard_normal((L.S * L.P, 12)).astype(np.float32)
+    unit = O.unit_features(dino)
+    for i in [L.n_special, L.V + L.n_special + 7, L.N - 1]:
+        s_i, loc = O.token_parts(L, i)
+        a = s_i * L.P + loc - L.n_special
+        for k in (1, 3, L.P):
+            got = O.token_topk_row(L, unit, i, k)
+            for sv in range(L.S):
+                cos = [float(np.float32(np.dot(dino[a], dino[sv * L.P + p]) /
+                                        (np.linalg.norm(dino[a].astype(np.float64)) *
+                                         np.linalg.norm(dino[sv * L.P + p].astype(np.float64)))))
+                       for p in range(L.P)]
+                want = sorted(range(L.P), key=lambda p: (-cos[p], p))[:k]
+                assert got[sv].tolist() == want
+            assert got[s_i][0] == a - s_i * L.P  # a token is most similar to itself
+    hc = HeadCfg(TOKEN, k=L.P)
+    sel = O.select(L, [hc], None, None, dino)
+    for i in (0, L.n_special, L.N - 1):
+        assert O.key_set(L, hc, sel, 0, i).tolist() == list(range(L.N))
+    hc = HeadCfg(TOKEN, k=2)
+    sel = O.select(L, [hc], None, None, dino)
+    assert O.kept_pairs(L, hc, sel, 0) == sum(len(O.key_set(L, hc, sel, 0, i)) for i in range(L.N))
