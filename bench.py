@@ -38,10 +38,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attention launch on this workload, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on: a changed kernel reports null until it is re-captured.
-# Taken on the S=32-view call (189,872,896 + 70,550,272 bytes) and scaled to the
+# Taken on the S=32-view call (189,911,040 + 70,724,864 bytes) and scaled to the
 # S=100-view call by the token count (137,400 / 43,968): Q/K/V/O bytes grow with N.
-ATTN_TRAFFIC = {"kernel_source_sha256": "48c5abe8d29cab010bf72696f3cdb51a3362cea7328086c5c4a0f762308e6a2a",
-                "bytes_per_launch": round((189872896 + 70550272) * 137400 / 43968), "workload": "s100"}
+ATTN_TRAFFIC = {"kernel_source_sha256": "e2e396f8a6f69c8e77ff2033b0fd65a1af3eff36fd75a61f75592c953a9fcd45",
+                "bytes_per_launch": round((189911040 + 70724864) * 137400 / 43968), "workload": "s100"}
 
 
 def kernel_source_sha256():
