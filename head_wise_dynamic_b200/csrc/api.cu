@@ -146,7 +146,7 @@ saf3r_status check_cfg(const Dims& d, const saf3r_head_cfg* cfg, int H) {
         break;
       case SAF3R_TOKEN:
         if (c.k < 1 || c.k > d.P) return SAF3R_ERR_INVALID;
-        if (d.dino_dim > kTokenMaxDim || token_topk_smem_bytes(d.P, c.k) > 200 * 1024) return SAF3R_ERR_UNSUPPORTED;
+        if (d.dino_dim > kTokenMaxDim || token_rank_smem_bytes(d.P, c.k) > 200 * 1024) return SAF3R_ERR_UNSUPPORTED;
         break;
       default:
         return SAF3R_ERR_INVALID;
@@ -526,6 +526,18 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
 
 }  // namespace
 
+bool saf3r::make_map_f16_rows(CUtensorMap* m, const void* base, long long rows, int cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows < 1 ? 1 : rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ======================================================================== C ABI
 extern "C" {
 
@@ -606,6 +618,9 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   sp.S = d.S;
   sp.tok_kmax = cl.tok_kmax;
   sp.tok_off = cl.tok_off;
+  sp.num_sms = dev.sms;
+  sp.err = dev.err;
+  sp.wait_budget = kWaitBudget;
   CacheHeader& hd = sp.header;
   std::memset(&hd, 0, sizeof(hd));
   hd.magic = kCacheMagic;

@@ -119,6 +119,17 @@ struct TokenAttnParams {
   int* err;
 };
 
+// Tensor-core cosines of the token-wise selection (token_sim.cu): scores[r][c] (fp16, row
+// stride ld halves) = unit16[r0 + r] . unit16[c] for r < rows, c < ld, over n_kc 64-feature slices.
+struct TokenSimParams {
+  int r0, rows;          // first query row of this chunk, rows in the chunk
+  int n_rb, n_ct, n_kc;  // 128-row blocks, 256-column tiles, 64-feature slices
+  long long ld;          // score row stride in halves (a multiple of 8, >= the candidate rows)
+  uint16_t* scores;
+  int* err;
+  long long wait_budget;
+};
+
 // Selection plan (select.cu).
 struct SelectPlan {
   int N, V, ns, P, T, dim;
@@ -132,6 +143,9 @@ struct SelectPlan {
   int S;
   int tok_kmax;             // token-wise heads: widest per-frame budget (0 = none)
   long long tok_off;
+  int num_sms;
+  int* err;                 // device error word (bounded waits of the tensor-core kernels)
+  long long wait_budget;
   CacheHeader header;
 };
 
@@ -168,7 +182,11 @@ cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tmQ, const 
                              const CUtensorMap& tmV, const CUtensorMap& tmQC, const CUtensorMap& tmKC,
                              const CUtensorMap& tmVC, int num_sms, cudaStream_t stream);
 size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows);
-size_t token_topk_smem_bytes(int P, int kmax);
+size_t token_rank_smem_bytes(int P, int kmax);
+size_t token_sim_smem_bytes();
+cudaError_t launch_token_sim(const TokenSimParams& p, const CUtensorMap& tm, int num_sms, cudaStream_t stream);
+// [rows][cols] fp16, 64 x 128 boxes, 128-byte swizzle, zero fill out of range (api.cu)
+bool make_map_f16_rows(CUtensorMap* m, const void* base, long long rows, int cols);
 cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_t* k, const float* dino,
                           int32_t* cache, uint8_t* ws, cudaStream_t stream, int* n_launch);
 cudaError_t launch_cache_check(const void* cache, uint64_t hash, int N, int T, int* ok, int* err,

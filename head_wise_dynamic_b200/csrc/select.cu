@@ -9,6 +9,7 @@
 //    L2-normalised DINO features of its patch tokens; tiles are compared by
 //    cosine (fp64 dot of the normalised means); each query tile ranks all
 //    tiles, itself included, best first, ties to the lower tile index.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -505,10 +506,17 @@ __global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __rest
 
 // ---- token-wise DINO Top-K (section 4.1, "DINO Top-K Kernel": per query token, the Top-K most
 // similar tokens of every frame; section 5.1: K per frame)
+//
+// Three steps: unit features (fp32, and an fp16 copy zero-padded to a multiple of 64 features);
+// the fp16 cosines of a chunk of query rows against all patch tokens on the tensor cores
+// (token_sim.cu, within kTokScoreErr of the exact cosine); and, per query row and frame, the
+// ranking below, which recomputes exactly (fp64 dot, rounded to fp32) every candidate the
+// bound cannot rule out.
 
 // Unit DINO features, one warp per patch token: fp64 sum of squares, one scale in fp32.
 __global__ void __launch_bounds__(256) unit_features_kernel(const float* __restrict__ dino, int rows, int dim,
-                                                            float* __restrict__ unit) {
+                                                            float* __restrict__ unit, __half* __restrict__ unit16,
+                                                            int dim16) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= rows) return;
   const float* f = dino + static_cast<size_t>(warp) * dim;
@@ -517,35 +525,301 @@ __global__ void __launch_bounds__(256) unit_features_kernel(const float* __restr
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float inv = ss > 0.0 ? static_cast<float>(1.0 / sqrt(ss)) : 0.f;
-  for (int c = lane; c < dim; c += 32) unit[static_cast<size_t>(warp) * dim + c] = f[c] * inv;
+  for (int c = lane; c < dim16; c += 32) {
+    const float u = c < dim ? f[c] * inv : 0.f;
+    if (c < dim) unit[static_cast<size_t>(warp) * dim + c] = u;
+    unit16[static_cast<size_t>(warp) * dim16 + c] = __float2half_rn(u);
+  }
 }
 
-// Eight query patch tokens per block; for every frame s the fp32 cosines against the frame's P
-// patch tokens, then each warp ranks its query's frame exactly (as the tile form) and writes
-// the kmax best patch indices to lists[(a * S + s) * kmax + rank], a = query's feature row.
-__global__ void __launch_bounds__(256) token_topk_kernel(const float* __restrict__ unit, int S, int P, int dim,
-                                                         int kmax, int32_t* __restrict__ lists) {
-  extern __shared__ uint8_t tk_smem[];
-  float* cs = reinterpret_cast<float*>(tk_smem);                               // [8][P]
-  int* hist = reinterpret_cast<int*>(cs + static_cast<size_t>(kTkRows) * P);  // [8 warps][256]
-  int* sel_idx = hist + 8 * 256;                                               // [8 warps][kmax]
-  uint32_t* sel_key = reinterpret_cast<uint32_t*>(sel_idx + 8 * kmax);         // [8 warps][kmax]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rows = S * P;
-  const int a0 = blockIdx.x * kTkRows;
-  const int nr = min(kTkRows, rows - a0);
-  float4 q[kTkRows][kTkChunks];
-  load_row_slices(unit, a0, nr, dim, lane, q);
-  for (int s = 0; s < S; ++s) {
-    const float* cand = unit + static_cast<size_t>(s) * P * dim;
-    dots_fp32(q, cand, P, dim, nr, cs, P, warp, lane);
-    __syncthreads();
-    if (warp < nr)
-      rank_row_exact(cs + static_cast<size_t>(warp) * P, P, kmax, q, warp, cand, dim, hist + warp * 256,
-                     sel_idx + warp * kmax, sel_key + warp * kmax, lane,
-                     lists + (static_cast<size_t>(a0 + warp) * S + s) * kmax);
-    __syncthreads();
+constexpr float kTokScoreErr = 2e-3f;  // |tensor-core fp16 score - exact cosine| (bound in token_sim.cu)
+constexpr int kTokCap = 64;            // candidates of one (query, frame) the short ranking takes
+
+// This lane's slice of unit vector `row` (features 128c + 4 lane .. +3).
+__device__ __forceinline__ void load_one_slice(const float* __restrict__ vec, int row, int dim, int lane,
+                                               float4 (&q)[kTkChunks]) {
+#pragma unroll
+  for (int c = 0; c < kTkChunks; ++c) {
+    const int d = 128 * c + 4 * lane;
+    q[c] = d < dim ? ld_f4(vec + static_cast<size_t>(row) * dim + d) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+
+// fp64 dot of the lane slices q with candidate row fv, summed over the warp (every lane gets
+// the same value: a butterfly adds the same two operands on both sides of each exchange).
+__device__ __forceinline__ double exact_dot(const float4 (&q)[kTkChunks], const float* __restrict__ fv, int dim,
+                                           int lane) {
+  double acc = 0.0;
+#pragma unroll
+  for (int c = 0; c < kTkChunks; ++c) {
+    const int d = 128 * c + 4 * lane;
+    if (d < dim) {
+      const float4 b = ld_f4(fv + d);
+      acc = fma(static_cast<double>(q[c].x), static_cast<double>(b.x), acc);
+      acc = fma(static_cast<double>(q[c].y), static_cast<double>(b.y), acc);
+      acc = fma(static_cast<double>(q[c].z), static_cast<double>(b.z), acc);
+      acc = fma(static_cast<double>(q[c].w), static_cast<double>(b.w), acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
+struct TokWarpSmem {
+  float* row;       // [P] approximate scores (general ranking)
+  int* hist;        // [256]
+  int* widx;        // [kmax]
+  uint32_t* wkey;   // [kmax]
+  int* cidx;        // [kTokCap] candidate patch indices (ascending)
+  float* cval;      // [kTokCap] their approximate scores
+  uint32_t* ckey;   // [kTokCap] order keys of their exact scores
+};
+
+// General ranking of one (query, frame): every candidate within 2 * kTokScoreErr of the
+// approximate kmax-th score gets its exact value, then the whole frame is ranked.
+__device__ void token_rank_general(const __half* __restrict__ seg, int P, int kmax, const float4 (&q)[kTkChunks],
+                                   const float* __restrict__ cand, int dim, const TokWarpSmem& w, int lane,
+                                   int32_t* __restrict__ out) {
+  for (int v = lane; v < P; v += 32) w.row[v] = __half2float(seg[v]);
+  __syncwarp();
+  uint32_t prefix;
+  int remaining;
+  warp_radix_kth(w.row, P, kmax, w.hist, lane, prefix, remaining);
+  const float thr = key_value(prefix) - 2.f * kTokScoreErr;
+  for (int v0 = 0; v0 < P; v0 += 32) {
+    const int v = v0 + lane;
+    uint32_t todo = __ballot_sync(0xffffffffu, v < P && w.row[v] >= thr);
+    while (todo) {
+      const int bit = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const double e = exact_dot(q, cand + static_cast<size_t>(v0 + bit) * dim, dim, lane);
+      if (lane == 0) w.row[v0 + bit] = static_cast<float>(e);
+    }
+  }
+  __syncwarp();
+  warp_rank_row(w.row, P, kmax, w.hist, w.widx, w.wkey, lane, out);
+}
+
+// Two fp64 dots at once (both rows' loads in flight together); see exact_dot.
+__device__ __forceinline__ void exact_dot2(const float4 (&q)[kTkChunks], const float* __restrict__ f1,
+                                           const float* __restrict__ f2, int dim, int lane, double& e1, double& e2) {
+  float4 b1[kTkChunks], b2[kTkChunks];
+#pragma unroll
+  for (int c = 0; c < kTkChunks; ++c) {
+    const int d = 128 * c + 4 * lane;
+    b1[c] = d < dim ? ld_f4(f1 + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+    b2[c] = d < dim ? ld_f4(f2 + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  double a1 = 0.0, a2 = 0.0;
+#pragma unroll
+  for (int c = 0; c < kTkChunks; ++c) {
+    const double qx = q[c].x, qy = q[c].y, qz = q[c].z, qw = q[c].w;
+    a1 = fma(qx, static_cast<double>(b1[c].x), a1);
+    a2 = fma(qx, static_cast<double>(b2[c].x), a2);
+    a1 = fma(qy, static_cast<double>(b1[c].y), a1);
+    a2 = fma(qy, static_cast<double>(b2[c].y), a2);
+    a1 = fma(qz, static_cast<double>(b1[c].z), a1);
+    a2 = fma(qz, static_cast<double>(b2[c].z), a2);
+    a1 = fma(qw, static_cast<double>(b1[c].w), a1);
+    a2 = fma(qw, static_cast<double>(b2[c].w), a2);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+    a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+  }
+  e1 = a1;
+  e2 = a2;
+}
+
+// The 8 scores of 16-byte chunk c of a score row (fp32) and which of them lie in the frame
+// [e0, e0 + P) (bit j for score j; all 8 for a chunk inside the frame).
+__device__ __forceinline__ uint32_t chunk_scores(const uint4 w, int c, int e0, int P, float (&v)[8]) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+  const int j0 = 8 * c - e0;  // frame index of v[0]
+  uint32_t valid = 0xFFu;
+  if (j0 < 0 || j0 + 8 > P) {
+    valid = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = j0 + j >= 0 && j0 + j < P;
+      valid |= static_cast<uint32_t>(in) << j;
+      if (!in) v[j] = -INFINITY;
+    }
+  }
+  return valid;
+}
+
+// Ranking of one (query, frame) from its approximate scores: frame s occupies elements
+// [e0, e0 + P) of the score row srow (16-byte aligned).
+//
+// With a = approximate score, e = exact score, |a - e| <= b = kTokScoreErr, A_k = the kmax-th
+// largest a and E_k the kmax-th largest e: A_k <= E_k + b (of the kmax largest a, one at least
+// has e <= E_k), so every key of the exact Top-kmax has a >= E_k - b >= A_k - 2b, and every key
+// with a < A_k - 2b has e < E_k.  The kmax-th largest of the 32 lane maxima t0 is <= A_k, so
+// D = {a >= t0 - 2b} holds every such key; when D fits kTokCap the short path finds A_k inside D,
+// recomputes C = {a >= A_k - 2b} exactly and ranks C (exact value descending, index ascending),
+// which is the frame's exact ranking.  Otherwise (kmax > 32, or more than kTokCap keys in D)
+// the general ranking runs.
+__device__ void token_rank_frame(const __half* __restrict__ srow, int e0, int P, int kmax,
+                                 const float4 (&q)[kTkChunks], const float* __restrict__ cand, int dim,
+                                 const TokWarpSmem& w, int lane, int32_t* __restrict__ out) {
+  const float band = 2.f * kTokScoreErr;
+  const uint4* row4 = reinterpret_cast<const uint4*>(srow);
+  const int cb = e0 >> 3, ce = (e0 + P + 7) >> 3;
+  bool general = kmax > 32;
+  int n = 0;
+  if (!general) {
+    float m = -INFINITY;
+    for (int c = cb + lane; c < ce; c += 32) {
+      float v[8];
+      chunk_scores(__ldg(row4 + c), c, e0, P, v);
+      m = fmaxf(m, fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7]))));
+    }
+    // bitonic sort of the 32 lane maxima, descending: lane kmax-1 then holds the kmax-th largest
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const float y = __shfl_xor_sync(0xffffffffu, m, j);
+        m = (((lane & j) == 0) == ((lane & k) == 0)) ? fmaxf(m, y) : fminf(m, y);
+      }
+    const float thr = __shfl_sync(0xffffffffu, m, kmax - 1) - band;  // -inf when fewer keys than lanes hold
+    for (int c0 = cb; c0 < ce; c0 += 32) {
+      const int c = c0 + lane;
+      float v[8];
+      uint32_t bits = 0;
+      if (c < ce) {
+        const uint32_t valid = chunk_scores(__ldg(row4 + c), c, e0, P, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) bits |= static_cast<uint32_t>(v[j] >= thr) << j;
+        bits &= valid;
+      }
+      const int cnt = __popc(bits);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int pos = n + incl - cnt;
+      if (bits) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if ((bits >> j) & 1u) {
+            if (pos < kTokCap) {
+              w.cidx[pos] = 8 * c + j - e0;
+              w.cval[pos] = v[j];
+            }
+            ++pos;
+          }
+      }
+      n += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    general = n > kTokCap || n < kmax;
+  }
+  if (general) {
+    __syncwarp();
+    token_rank_general(srow + e0, P, kmax, q, cand, dim, w, lane, out);
+    return;
+  }
+  __syncwarp();
+  // A_k: the kmax-th largest approximate score of D (ties by position)
+  float ak = 0.f;
+  {
+    bool hit = false;
+    float hv = 0.f;
+    for (int i = lane; i < n; i += 32) {
+      const float ai = w.cval[i];
+      int r = 0;
+      for (int j = 0; j < n; ++j) {
+        const float aj = w.cval[j];
+        r += (aj > ai) || (aj == ai && j < i);
+      }
+      if (r == kmax - 1) {
+        hit = true;
+        hv = ai;
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, hit)) - 1;
+    ak = __shfl_sync(0xffffffffu, hv, src);
+  }
+  const float cthr = ak - band;
+  // exact values of C, two candidates at a time
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int i = i0 + lane;
+    uint32_t todo = __ballot_sync(0xffffffffu, i < n && w.cval[i] >= cthr);
+    while (todo) {
+      const int b1 = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int b2 = todo ? __ffs(todo) - 1 : b1;
+      if (todo) todo &= todo - 1;
+      double e1, e2;
+      exact_dot2(q, cand + static_cast<size_t>(w.cidx[i0 + b1]) * dim, cand + static_cast<size_t>(w.cidx[i0 + b2]) * dim,
+                 dim, lane, e1, e2);
+      if (lane == 0) {
+        w.ckey[i0 + b1] = order_key(static_cast<float>(e1));
+        if (b2 != b1) w.ckey[i0 + b2] = order_key(static_cast<float>(e2));
+      }
+    }
+  }
+  __syncwarp();
+  // rank C: exact value descending, then patch index ascending
+  for (int i = lane; i < n; i += 32) {
+    if (w.cval[i] < cthr) continue;
+    const uint32_t ki = w.ckey[i];
+    const int vi = w.cidx[i];
+    int r = 0;
+    for (int j = 0; j < n; ++j) {
+      if (w.cval[j] < cthr) continue;
+      const uint32_t kj = w.ckey[j];
+      r += (kj > ki) || (kj == ki && w.cidx[j] < vi);
+    }
+    if (r < kmax) out[r] = vi;
+  }
+  __syncwarp();
+}
+
+// One warp per query row of the chunk; frames in turn.  lists[(a * S + s) * kmax + rank] =
+// patch index of rank `rank` in frame s for feature row a = r0 + row.
+__global__ void __launch_bounds__(256, 3) token_rank_kernel(const __half* __restrict__ scores, long long ld, int r0,
+                                                         int rows, const float* __restrict__ unit, int S, int P,
+                                                         int dim, int kmax, int32_t* __restrict__ lists) {
+  extern __shared__ uint8_t tr_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  TokWarpSmem w;
+  {
+    float* rows_f = reinterpret_cast<float*>(tr_smem);
+    int* hist = reinterpret_cast<int*>(rows_f + static_cast<size_t>(8) * P);
+    int* cidx = hist + 8 * 256;
+    float* cval = reinterpret_cast<float*>(cidx + 8 * kTokCap);
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(cval + 8 * kTokCap);
+    int* widx = reinterpret_cast<int*>(ckey + 8 * kTokCap);
+    uint32_t* wkey = reinterpret_cast<uint32_t*>(widx + 8 * kmax);
+    w.row = rows_f + static_cast<size_t>(warp) * P;
+    w.hist = hist + warp * 256;
+    w.cidx = cidx + warp * kTokCap;
+    w.cval = cval + warp * kTokCap;
+    w.ckey = ckey + warp * kTokCap;
+    w.widx = widx + warp * kmax;
+    w.wkey = wkey + warp * kmax;
+  }
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;
+  const int a = r0 + row;
+  float4 q[kTkChunks];
+  load_one_slice(unit, a, dim, lane, q);
+  const __half* srow = scores + static_cast<size_t>(row) * ld;
+  for (int s = 0; s < S; ++s)
+    token_rank_frame(srow, s * P, P, kmax, q, unit + static_cast<size_t>(s) * P * dim, dim, w, lane,
+                     lists + (static_cast<size_t>(a) * S + s) * kmax);
 }
 
 // ---- query-tile grouping of the correspondence heads (a scheduling aid, cached with the indices)
@@ -672,6 +946,32 @@ __global__ void cache_header_kernel(CacheHeader h, CacheHeader* dst) {
 
 }  // namespace
 
+// Workspace of the token-wise selection, after everything else: fp32 unit features [R][dim],
+// fp16 unit features [R][dim16] (dim16 = dim rounded up to 64, zero-padded), and fp16 scores of
+// one chunk of query rows [rows][ld] (ld = R rounded up to 8; chunks of at most ~1 GiB).
+struct TokWs {
+  int dim16;
+  long long ld;
+  int chunk_rows;
+  size_t unit, unit16, scores, end;  // byte offsets from the token part's start
+};
+
+constexpr size_t kTokScoreBudget = size_t(1) << 30;
+
+TokWs token_ws(long long R, int dim) {
+  TokWs t;
+  t.dim16 = (dim + 63) / 64 * 64;
+  t.ld = (R + 7) / 8 * 8;
+  long long rows = static_cast<long long>(kTokScoreBudget / (static_cast<size_t>(t.ld) * 2)) / 128 * 128;
+  if (rows < 128) rows = 128;
+  t.chunk_rows = static_cast<int>(rows < R ? rows : R);
+  t.unit = 0;
+  t.unit16 = (static_cast<size_t>(R) * dim * sizeof(float) + 255) & ~size_t(255);
+  t.scores = (t.unit16 + static_cast<size_t>(R) * t.dim16 * 2 + 255) & ~size_t(255);
+  t.end = t.scores + static_cast<size_t>(t.chunk_rows) * t.ld * 2;
+  return t;
+}
+
 size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows) {
   size_t b = 0;
   b += static_cast<size_t>(n_probe) * kProbePartials * kD * sizeof(double);
@@ -687,12 +987,13 @@ size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, lon
     b += static_cast<size_t>(T) * sizeof(int32_t);                      // sorted tiles
   }
   b = ((b + 255) & ~size_t(255)) + 256;
-  b += static_cast<size_t>(tok_rows) * dim * sizeof(float);  // unit features of the token-wise heads
+  if (tok_rows > 0) b += token_ws(tok_rows, dim).end;
   return b;
 }
 
-size_t token_topk_smem_bytes(int P, int kmax) {
-  return sizeof(float) * static_cast<size_t>(kTkRows) * P + sizeof(int) * (8 * 256 + 16 * static_cast<size_t>(kmax));
+size_t token_rank_smem_bytes(int P, int kmax) {
+  return 8 * (sizeof(float) * static_cast<size_t>(P) + sizeof(int) * 256 + 3 * sizeof(int) * kTokCap +
+              2 * sizeof(int) * static_cast<size_t>(kmax));
 }
 
 
@@ -788,18 +1089,40 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
     }
   }
   if (sp.tok_kmax > 0) {
-    // unit features after everything else of the workspace
-    float* unit = reinterpret_cast<float*>(ws + select_workspace_bytes(sp.n_probe, sp.N, sp.T, sp.dim,
-                                                                        sp.corr_kmax > 0, 0));
-    const int rows = sp.S * sp.P;
-    unit_features_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(dino, rows, sp.dim, unit);
-    const size_t smem = token_topk_smem_bytes(sp.P, sp.tok_kmax);
-    cudaError_t e =
-        cudaFuncSetAttribute(token_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    // the token part of the workspace, after everything else
+    uint8_t* base = ws + select_workspace_bytes(sp.n_probe, sp.N, sp.T, sp.dim, sp.corr_kmax > 0, 0);
+    const long long R = static_cast<long long>(sp.S) * sp.P;
+    const TokWs tw = token_ws(R, sp.dim);
+    float* unit = reinterpret_cast<float*>(base + tw.unit);
+    __half* unit16 = reinterpret_cast<__half*>(base + tw.unit16);
+    __half* scores = reinterpret_cast<__half*>(base + tw.scores);
+    unit_features_kernel<<<static_cast<unsigned>((R + 7) / 8), 256, 0, stream>>>(dino, static_cast<int>(R), sp.dim,
+                                                                                 unit, unit16, tw.dim16);
+    ++*n_launch;
+    CUtensorMap tm;
+    if (!make_map_f16_rows(&tm, unit16, R, tw.dim16)) return cudaErrorInvalidValue;
+    const size_t rsmem = token_rank_smem_bytes(sp.P, sp.tok_kmax);
+    cudaError_t e = cudaFuncSetAttribute(token_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(rsmem));
     if (e != cudaSuccess) return e;
-    token_topk_kernel<<<(rows + kTkRows - 1) / kTkRows, 256, smem, stream>>>(unit, sp.S, sp.P, sp.dim, sp.tok_kmax,
-                                                                             cache + sp.tok_off);
-    *n_launch += 2;
+    for (long long r0 = 0; r0 < R; r0 += tw.chunk_rows) {
+      const int rows = static_cast<int>(R - r0 < tw.chunk_rows ? R - r0 : tw.chunk_rows);
+      TokenSimParams tp;
+      tp.r0 = static_cast<int>(r0);
+      tp.rows = rows;
+      tp.n_rb = (rows + 127) / 128;
+      tp.n_ct = static_cast<int>((R + 255) / 256);
+      tp.n_kc = tw.dim16 / 64;
+      tp.ld = tw.ld;
+      tp.scores = reinterpret_cast<uint16_t*>(scores);
+      tp.err = sp.err;
+      tp.wait_budget = sp.wait_budget;
+      e = launch_token_sim(tp, tm, sp.num_sms, stream);
+      if (e != cudaSuccess) return e;
+      token_rank_kernel<<<(rows + 7) / 8, 256, rsmem, stream>>>(scores, tw.ld, static_cast<int>(r0), rows, unit, sp.S,
+                                                                sp.P, sp.dim, sp.tok_kmax, cache + sp.tok_off);
+      *n_launch += 2;
+    }
   }
   return cudaGetLastError();
 }

@@ -126,10 +126,12 @@ size_t saf3r_profile_workspace_bytes(const saf3r_layout* layout, const saf3r_hea
  *   - TOKEN heads: L2-normalised DINO features; for every patch query and
  *     every frame, the frame's patch tokens ranked by cosine (own token
  *     included; ties to the lower patch index); the lists are cached.
- *     The cosines are formed in fp32 and every candidate within the fp32
- *     error bound of the k-th value is recomputed exactly (fp64), so the
- *     ranking is that of the fp64 cosines rounded to fp32.  Needs
- *     dino_dim <= 384 (SAF3R_ERR_UNSUPPORTED otherwise).
+ *     The cosines are formed on the tensor cores (fp16 features, fp32
+ *     accumulation, fp16 scores: within 2e-3 of the exact cosine) and every
+ *     candidate within twice that bound of the k-th score is recomputed
+ *     exactly (fp64), so the ranking is that of the fp64 cosines rounded to
+ *     fp32.  The workspace then holds the fp16 scores of up to 1 GiB of query
+ *     rows at a time.  Needs dino_dim <= 384 (SAF3R_ERR_UNSUPPORTED otherwise).
  *   - POSITION, SCAN and DENSE heads need no cached state (a HYBRID head's
  *     lattice neither).
  * q, k: bf16 [H][N][d]; dino: fp32 patch features, or NULL when no head is

@@ -227,6 +227,27 @@ def test_token_heads_all_rows(name):
             assert int(pairs[h]) == sum(O.kept_count(case.L, hc, sel, h, i) for i in range(case.L.N))
 
 
+@pytest.mark.parametrize("n_feat", [2, 5])
+def test_token_heads_tied_features(n_feat):
+    """Every patch takes one of n_feat DINO features, so a query's scores tie in large groups:
+    with 2 features a frame's candidates overflow the short ranking (the general ranking runs),
+    with 5 the short ranking sees whole tie groups; k = 40 always takes the general ranking.
+    Ties go to the lower patch index on both sides, so the lists must be identical."""
+    case = Case(_custom(3, 12, [HeadCfg(TOKEN, k=16), HeadCfg(TOKEN, k=5), HeadCfg(TOKEN, k=40),
+                                HeadCfg(SCAN, stride=4, phase=1)]))
+    L = case.L
+    rng = np.random.default_rng(40 + n_feat)
+    base = rng.standard_normal((n_feat, L.dino_dim)).astype(np.float32)
+    case.dino = torch.from_numpy(np.ascontiguousarray(base[rng.integers(0, n_feat, size=L.S * L.P)])).cuda()
+    heads = case.wl.heads
+    att, out = run_gpu(case, heads)
+    sel = oracle_select(case, heads)
+    exact = check_selection(case, heads, att, sel)
+    exact.update(_check_token_heads(case, heads, att, sel, np.arange(L.N)))
+    assert all(exact[h] for h in range(3)), exact
+    check_rows(case, heads, sel, out, lambda h: np.arange(L.N), exact)
+
+
 def test_s32_token_heads_sampled_rows(s32):
     """Per-frame Top-16 token-wise heads on the S=32 layer (the other heads as configured)."""
     heads = [HeadCfg(TOKEN, k=16)] * 4 + list(s32.wl.heads[4:])
