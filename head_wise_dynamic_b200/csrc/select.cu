@@ -752,10 +752,30 @@ __device__ void token_rank_frame(const __half* __restrict__ srow, int e0, int P,
     ak = __shfl_sync(0xffffffffu, hv, src);
   }
   const float cthr = ak - band;
-  // exact values of C, two candidates at a time
-  for (int i0 = 0; i0 < n; i0 += 32) {
-    const int i = i0 + lane;
-    uint32_t todo = __ballot_sync(0xffffffffu, i < n && w.cval[i] >= cthr);
+  // A key of C whose approximate score is more than `band` away from every other key of C has
+  // the same order against each of them by exact value (|a - e| <= b on both sides), so only the
+  // keys with a neighbour within `band` (ambiguous) need their exact value; ckey = 0 (no real
+  // value has that order key) marks the others, which the ranking then orders by a.
+  bool amb[2] = {false, false};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = lane + 32 * h;
+    if (i < n) {
+      const float ai = w.cval[i];
+      if (ai >= cthr)
+        for (int j = 0; j < n; ++j) {
+          const float aj = w.cval[j];
+          amb[h] |= j != i && aj >= cthr && fabsf(aj - ai) <= band;
+        }
+      w.ckey[i] = 0u;
+    }
+  }
+  __syncwarp();
+  // exact values of the ambiguous keys, two at a time
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i0 = 32 * h;
+    uint32_t todo = __ballot_sync(0xffffffffu, amb[h]);
     while (todo) {
       const int b1 = __ffs(todo) - 1;
       todo &= todo - 1;
@@ -773,14 +793,16 @@ __device__ void token_rank_frame(const __half* __restrict__ srow, int e0, int P,
   __syncwarp();
   // rank C: exact value descending, then patch index ascending
   for (int i = lane; i < n; i += 32) {
-    if (w.cval[i] < cthr) continue;
+    const float ai = w.cval[i];
+    if (ai < cthr) continue;
     const uint32_t ki = w.ckey[i];
     const int vi = w.cidx[i];
     int r = 0;
     for (int j = 0; j < n; ++j) {
-      if (w.cval[j] < cthr) continue;
+      const float aj = w.cval[j];
+      if (aj < cthr || j == i) continue;
       const uint32_t kj = w.ckey[j];
-      r += (kj > ki) || (kj == ki && w.cidx[j] < vi);
+      r += (ki != 0u && kj != 0u) ? ((kj > ki) || (kj == ki && w.cidx[j] < vi)) : (aj > ai);
     }
     if (r < kmax) out[r] = vi;
   }
