@@ -102,19 +102,19 @@ def stride_set(L, stride: int, phase: int) -> np.ndarray:
     return j[keep]
 
 
-def probe_mean(Qh: np.ndarray) -> np.ndarray:
+def probe_mean(Qh: np.ndarray, accum=np.float64) -> np.ndarray:
     """Mean query over all N queries (section 4.3, "Query-Probe Top-K Kernel"):
-    qbar = (1/N) sum_i q_i, summed in fp64 and rounded once to fp32."""
-    q = np.asarray(Qh, dtype=np.float64)
-    return (q.sum(axis=0) / q.shape[0]).astype(np.float32)
+    qbar = (1/N) sum_i q_i, summed in fp64 (or `accum`) and rounded once to fp32."""
+    q = np.asarray(Qh, dtype=accum)
+    return (q.sum(axis=0) / accum(q.shape[0])).astype(np.float32)
 
 
-def probe_scores(qbar32: np.ndarray, Kh: np.ndarray) -> np.ndarray:
-    """Probe score of every key, qbar K^T / sqrt(D) (section 4.3), in fp64 and
-    rounded to fp32 (the precision the selection is taken in)."""
-    k = np.asarray(Kh, dtype=np.float64)
+def probe_scores(qbar32: np.ndarray, Kh: np.ndarray, accum=np.float64) -> np.ndarray:
+    """Probe score of every key, qbar K^T / sqrt(D) (section 4.3), in fp64 (or
+    `accum`) and rounded to fp32 (the precision the selection is taken in)."""
+    k = np.asarray(Kh, dtype=accum)
     d = k.shape[1]
-    return ((k @ qbar32.astype(np.float64)) / math.sqrt(d)).astype(np.float32)
+    return ((k @ qbar32.astype(accum)) / accum(math.sqrt(d))).astype(np.float32)
 
 
 def topk_desc(scores: np.ndarray, k: int, candidates: np.ndarray | None = None) -> np.ndarray:
@@ -137,14 +137,14 @@ def probe_set(L, probe_keys: np.ndarray) -> np.ndarray:
     return np.union1d(probe_keys, special_tokens(L)).astype(np.int64)
 
 
-def dino_tile_means(L, dino: np.ndarray) -> np.ndarray:
+def dino_tile_means(L, dino: np.ndarray, accum=np.float64) -> np.ndarray:
     """Block-wise DINO descriptors (section 4.3, "DINO Top-K Kernel", block-wise
     variant): for each flat 64-token tile t = [64t, 64t+64) of the token
     sequence, the mean over its patch tokens of the L2-normalised DINO features
-    (special tokens carry no DINO feature).  fp64 [T][dino_dim]."""
-    f = np.asarray(dino, dtype=np.float64)
+    (special tokens carry no DINO feature).  fp64 (or `accum`) [T][dino_dim]."""
+    f = np.asarray(dino, dtype=accum)
     f = f / np.linalg.norm(f, axis=1, keepdims=True)
-    out = np.zeros((L.T, f.shape[1]), dtype=np.float64)
+    out = np.zeros((L.T, f.shape[1]), dtype=accum)
     for t in range(L.T):
         toks = np.arange(t * L.tile, min((t + 1) * L.tile, L.N), dtype=np.int64)
         toks = toks[~is_special(L, toks)]
@@ -157,7 +157,8 @@ def dino_tile_means(L, dino: np.ndarray) -> np.ndarray:
 
 
 def tile_cosines(means: np.ndarray) -> np.ndarray:
-    """Cosine similarity between every pair of tile descriptors, fp64 -> fp32."""
+    """Cosine similarity between every pair of tile descriptors, in the descriptors'
+    precision (fp64 unless the selection runs with fp32 accumulation) -> fp32."""
     nrm = np.linalg.norm(means, axis=1)
     cos = (means @ means.T) / np.outer(nrm, nrm)
     return cos.astype(np.float32)
@@ -184,9 +185,9 @@ def corr_set(L, tiles: Sequence[int]) -> np.ndarray:
     return np.unique(np.concatenate(parts))
 
 
-def unit_features(dino: np.ndarray) -> np.ndarray:
-    """L2-normalised DINO features of the patch tokens, fp64 [S*P][dim]."""
-    f = np.asarray(dino, dtype=np.float64)
+def unit_features(dino: np.ndarray, accum=np.float64) -> np.ndarray:
+    """L2-normalised DINO features of the patch tokens, fp64 (or `accum`) [S*P][dim]."""
+    f = np.asarray(dino, dtype=accum)
     return f / np.linalg.norm(f, axis=1, keepdims=True)
 
 
@@ -258,22 +259,25 @@ class Selection:
         self.tile_cos: np.ndarray | None = None
 
 
-def select(L, heads, Q, K, dino) -> Selection:
-    """Build the dynamic index sets of one input (section 4.3)."""
+def select(L, heads, Q, K, dino, accum=np.float64) -> Selection:
+    """Build the dynamic index sets of one input (section 4.3).  `accum` = np.float32
+    runs every reduction in fp32 instead of fp64, to show that the index sets do not
+    hinge on the accumulation precision (they may differ only at near-ties of the
+    k-th score)."""
     sel = Selection()
     kt_max = 0
     for h, hc in enumerate(heads):
         if hc.kind == PROBE:
-            qbar = probe_mean(Q[h])
-            sc = probe_scores(qbar, K[h])
+            qbar = probe_mean(Q[h], accum)
+            sc = probe_scores(qbar, K[h], accum)
             sel.probe_scores[h] = sc
             sel.probe_keys[h] = probe_topk(L, sc, hc.k)
         elif hc.kind in (CORR, HYBRID):
             kt_max = max(kt_max, hc.k)
         elif hc.kind == TOKEN and sel.unit is None:
-            sel.unit = unit_features(dino)
+            sel.unit = unit_features(dino, accum)
     if kt_max > 0:
-        cos = tile_cosines(dino_tile_means(L, dino))
+        cos = tile_cosines(dino_tile_means(L, dino, accum))
         sel.tile_cos = cos
         sel.tile_rank = tile_topk(cos, kt_max)
     return sel

@@ -359,3 +359,32 @@ def test_token_topk_brute_force_and_counts():
     hc = HeadCfg(TOKEN, k=2)
     sel = O.select(L, [hc], None, None, dino)
     assert O.kept_pairs(L, hc, sel, 0) == sum(len(O.key_set(L, hc, sel, 0, i)) for i in range(L.N))
+
+
+# ---------------------------------------------------------------- precision of the selection
+def test_selection_stable_under_fp32_accumulation():
+    """Every reduction of the selection run in fp32 instead of fp64 gives the same index sets,
+    up to keys whose fp64 score lies within the acceptance band (1e-5 relative) of the k-th
+    score: the probe, tile and token Top-K sets do not hinge on the accumulation precision, so a
+    GPU that forms scores in fp32 and recomputes only near-ties exactly selects the same keys."""
+    from parity_util import check_token_lists, check_topk_set
+    from saf3r_synth import Scene, Workload, bf16_to_f32, qkv
+    L = Layout(S=8, g=16, H=4)
+    heads = [HeadCfg(PROBE, k=300), HeadCfg(CORR, k=6), HeadCfg(TOKEN, k=12), HeadCfg(SCAN, stride=4, phase=1)]
+    wl = Workload("fp32-accumulation", L, M=256, delta=11, D=128, heads=heads, seed=9)
+    scene = Scene(wl)
+    Q, K, _ = (bf16_to_f32(t) for t in qkv(scene, 0))
+    dino = scene.dino()
+    s64 = O.select(L, heads, Q, K, dino)
+    s32 = O.select(L, heads, Q, K, dino, accum=np.float32)
+    assert s32.unit.dtype == np.float32 and s32.tile_cos is not None
+    sc = s64.probe_scores[0]
+    check_topk_set(s32.probe_keys[0], O.topk_desc(sc, 308, O.patch_tokens(L)), sc, 300, "probe fp32")
+    for u in range(L.T):
+        check_topk_set(s32.tile_rank[u, :6], O.topk_desc(s64.tile_cos[u], 14), s64.tile_cos[u], 6, f"tile {u} fp32")
+    lists = np.zeros((L.S * L.P, L.S, 12), dtype=np.int64)
+    rows = [i for i in range(L.N) if O.token_parts(L, i)[1] >= L.n_special]
+    for i in rows:
+        s_i, loc = O.token_parts(L, i)
+        lists[s_i * L.P + loc - L.n_special] = O.token_topk_row(L, s32.unit, i, 12)
+    check_token_lists(lists, L, s64.unit, 12, rows, "token fp32")
