@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 import head_wise_dynamic_b200 as hw
-from saf3r_synth import WORKLOADS
+from saf3r_synth import CORR, PROBE, SCAN, TOKEN, WORKLOADS, HeadCfg
 
 
 def test_library_exports_every_declared_symbol():
@@ -113,3 +113,22 @@ def test_token_cfg_validation():
     cfg[2].k = 4
     L.dino_dim = 388  # beyond what the token-wise selection keeps in registers: unsupported
     assert hw.saf3r_cache_bytes(L, cfg) == 0
+
+
+@pytest.mark.parametrize("S", [4, 32, 100])
+def test_token_select_workspace_on_host(S):
+    """Token-wise heads add to the select workspace: fp32 and fp16 unit features of the R = S*P
+    patch tokens and the fp16 scores of one chunk of query rows, at most 1 GiB of them (every
+    chunk a multiple of 128 rows, or all R rows)."""
+    from saf3r_synth import Layout
+    L = hw.layout_of(Layout(S=S, g=37 if S > 4 else 16, H=4))
+    base = [HeadCfg(PROBE, k=64), HeadCfg(CORR, k=4), HeadCfg(SCAN, stride=4, phase=1), HeadCfg(SCAN, stride=8)]
+    tok = [HeadCfg(PROBE, k=64), HeadCfg(CORR, k=4), HeadCfg(TOKEN, k=16), HeadCfg(SCAN, stride=8)]
+    w0 = hw.saf3r_workspace_bytes(L, hw.cfg_array(base), hw.OP_SELECT)
+    w1 = hw.saf3r_workspace_bytes(L, hw.cfg_array(tok), hw.OP_SELECT)
+    R = L.S * L.grid_h * L.grid_w
+    ld = (R + 7) // 8 * 8
+    feats = R * L.dino_dim * 4 + R * ((L.dino_dim + 63) // 64 * 64) * 2
+    chunk = min(R, max(128, (1 << 30) // (2 * ld) // 128 * 128))
+    assert w1 - w0 >= feats + chunk * ld * 2
+    assert w1 - w0 <= feats + min(R * ld * 2, (1 << 30)) + 4096
