@@ -205,13 +205,19 @@ def token_topk_row(L, unit: np.ndarray, i: int, k: int) -> np.ndarray:
     return out
 
 
-def token_set(L, unit: np.ndarray, i: int, k: int) -> np.ndarray:
+def token_set(L, unit: np.ndarray, i: int, k: int, lists: np.ndarray | None = None) -> np.ndarray:
     """Key set of a token-wise correspondence head for query i: the per-frame Top-K patch tokens
-    plus every special token; a special-token query (no DINO feature) keeps every key."""
+    plus every special token; a special-token query (no DINO feature) keeps every key.
+    `lists` ([S*P][S][>=k] patch indices per query and frame) replaces the ranking when given:
+    a set that another ranking produced and that was found valid (equal to this one's up to keys
+    tied within the boundary band), whose attention is then evaluated exactly."""
     s_i, loc = token_parts(L, int(i))
     if loc < L.n_special:
         return np.arange(L.N, dtype=np.int64)
-    p = token_topk_row(L, unit, i, k)
+    if lists is None:
+        p = token_topk_row(L, unit, i, k)
+    else:
+        p = np.asarray(lists[s_i * L.P + (loc - L.n_special)], dtype=np.int64)[:, :k]
     toks = (np.arange(L.S, dtype=np.int64)[:, None] * L.V + L.n_special + p).ravel()
     return np.union1d(toks, special_tokens(L)).astype(np.int64)
 
@@ -257,6 +263,8 @@ class Selection:
         self.tile_rank: np.ndarray | None = None
         self.unit: np.ndarray | None = None  # unit DINO features (token-wise heads; their sets are computed per row)
         self.tile_cos: np.ndarray | None = None
+        # per token-wise head, given per-frame lists [S*P][S][k] that replace the ranking (see token_set)
+        self.token_lists: Dict[int, np.ndarray] = {}
 
 
 def select(L, heads, Q, K, dino, accum=np.float64) -> Selection:
@@ -298,7 +306,7 @@ def key_set(L, hc, sel: Selection, h: int, i: int) -> np.ndarray:
         # with uniform striding, i.e. the union of the two kept sets
         return np.union1d(corr_set(L, sel.tile_rank[i // L.tile, :hc.k]), stride_set(L, hc.stride, hc.phase))
     if hc.kind == TOKEN:
-        return token_set(L, sel.unit, i, hc.k)
+        return token_set(L, sel.unit, i, hc.k, sel.token_lists.get(h))
     if hc.kind == DENSE:
         return np.arange(L.N, dtype=np.int64)
     raise ValueError(hc.kind)

@@ -1,4 +1,6 @@
 """Comparison helpers of the GPU parity tests (test code only)."""
+import copy
+
 import numpy as np
 
 import oracle as O
@@ -69,3 +71,51 @@ def check_token_lists(gpu_lists, L, unit, k, rows, what):
             ranked = O.topk_desc(frame, min(L.P, k + 8))
             exact &= check_topk_set(gpu_lists[a, sv], ranked, frame, k, f"{what} row {int(i)} frame {sv}")
     return exact
+
+
+def selection_over_gpu_set(sel, L, h, hc, exported):
+    """The oracle selection with head h's index set replaced by the one the GPU built.
+
+    Only for a set that check_topk_set (or check_token_lists) accepted: it equals the oracle's
+    own set up to keys tied within the boundary band, so it is a valid result of the selection,
+    and the oracle then evaluates the exact softmax attention over it (section 4.1 of the SAF3R
+    paper: each row attends exactly to its kept keys).  Where several sets are correct, this
+    checks that the attention the GPU ran is the one over the set it chose."""
+    s = copy.copy(sel)
+    if hc.kind == O.PROBE:
+        s.probe_keys = dict(sel.probe_keys)
+        s.probe_keys[h] = np.sort(np.asarray(exported, dtype=np.int64))
+    elif hc.kind in (O.CORR, O.HYBRID):
+        s.tile_rank = np.asarray(exported, dtype=np.int64).reshape(L.T, hc.k)
+    elif hc.kind == O.TOKEN:
+        s.token_lists = dict(sel.token_lists)
+        s.token_lists[h] = np.asarray(exported, dtype=np.int64).reshape(L.S * L.P, L.S, hc.k)
+    else:
+        raise ValueError(f"head kind {hc.kind} has no exported set")
+    return s
+
+
+class HeadSelections:
+    """Per head, the selection its output rows are checked against: the oracle's own where the
+    GPU's set is identical to it, else the oracle over the GPU's accepted set.  `over_gpu` names
+    the heads of the second kind (printed by the tests)."""
+
+    def __init__(self, sel):
+        self.base = sel
+        self.per_head = {}
+        self.over_gpu = []
+
+    def accept(self, L, h, hc, exported, exact):
+        if exact:
+            self.per_head[h] = self.base
+        else:
+            self.per_head[h] = selection_over_gpu_set(self.base, L, h, hc, exported)
+            self.over_gpu.append(h)
+
+    def __getitem__(self, h):
+        return self.per_head.get(h, self.base)
+
+    def report(self, what):
+        if self.over_gpu:
+            print(f"{what}: heads {self.over_gpu} resolved a boundary tie differently; their rows "
+                  f"were checked over the GPU's accepted set")

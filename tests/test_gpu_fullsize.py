@@ -6,42 +6,41 @@ import pytest
 
 import oracle as O
 from saf3r_synth import WORKLOADS, Scene, bf16_to_f32, qkv, sample_rows
-from parity_util import check_probe, check_tiles, compare_outputs
+from parity_util import HeadSelections, check_probe, check_tiles, compare_outputs
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 
-def _check_layer(wl, att, scene, layer, rows_per_head, sel=None):
+def _check_layer(wl, att, scene, layer, rows_per_head, sels=None):
+    """One layer call: on the first call (sels None) every index set against the oracle, then the
+    sampled rows of every head against the oracle over that head's validated set."""
     import head_wise_dynamic_b200 as hw
     L = wl.layout
     q, k, v = qkv(scene, layer, device="cuda")
     Q, K, V = (bf16_to_f32(t) for t in (q, k, v))
-    if sel is None:
+    if sels is None:
         att.select(q, k, torch.from_numpy(scene.dino()).cuda())
-        sel = O.select(L, wl.heads, Q, K, scene.dino())
-        exact = {}
+        sels = HeadSelections(O.select(L, wl.heads, Q, K, scene.dino()))
         for h, hc in enumerate(wl.heads):
-            if hc.kind == 1:
-                exact[h] = check_probe(hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h), L, sel, h, hc.k,
-                                       f"probe head {h}")
-            elif hc.kind in (2, 5):  # correspondence and hybrid heads: ranked tiles
+            if hc.kind == O.PROBE:
+                keys = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h)
+                sels.accept(L, h, hc, keys, check_probe(keys, L, sels.base, h, hc.k, f"probe head {h}"))
+            elif hc.kind in (O.CORR, O.HYBRID):  # ranked tiles
                 ranked = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(L.T, hc.k)
-                exact[h] = check_tiles(ranked, sel, hc.k, f"tile head {h}")
-        sel.exact = exact
+                sels.accept(L, h, hc, ranked, check_tiles(ranked, sels.base, hc.k, f"tile head {h}"))
     att.out.fill_(float("nan"))
     out = att(q, k, v)
     torch.cuda.synchronize()
     hw.saf3r_check()
     o = out.float().cpu().numpy()
     for h, hc in enumerate(wl.heads):
-        if not sel.exact.get(h, True):
-            continue
         rows = sample_rows(wl, h, rows_per_head, seed_extra=layer)
-        ref = O.sparse_rows(L, hc, sel, h, Q[h], K[h], V[h], rows)
+        ref = O.sparse_rows(L, hc, sels[h], h, Q[h], K[h], V[h], rows)
         compare_outputs(o[h][rows], ref, f"layer {layer} head {h}")
+    sels.report(f"{wl.name} layer {layer}")
     assert np.isfinite(o).all(), "a row was not written"
-    return sel
+    return sels
 
 
 def test_s100_layer_and_cache_reuse():
@@ -49,9 +48,9 @@ def test_s100_layer_and_cache_reuse():
     wl = WORKLOADS["s100"]
     scene = Scene(wl)
     att = hw.SparseGlobalAttention(wl.layout, wl.heads)  # bf16 output, as timed
-    sel = _check_layer(wl, att, scene, 0, 2048)
+    sels = _check_layer(wl, att, scene, 0, 2048)
     # a later layer call with fresh Q/K/V reuses the cached sets
-    _check_layer(wl, att, scene, wl.calls - 1, 256, sel=sel)
+    _check_layer(wl, att, scene, wl.calls - 1, 256, sels=sels)
 
 
 def test_s200_layer():

@@ -7,7 +7,7 @@ import pytest
 import oracle as O
 from saf3r_synth import (CORR, DENSE, HYBRID, POSITION, PROBE, SCAN, TOKEN, WORKLOADS, HeadCfg, Layout, Scene,
                          Workload, bf16_to_f32, qkv, sample_rows)
-from parity_util import check_probe, check_tiles, check_token_lists, compare_outputs
+from parity_util import HeadSelections, check_probe, check_tiles, check_token_lists, compare_outputs
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -46,26 +46,29 @@ def oracle_select(case, heads):
 
 
 def check_selection(case, heads, att, sel):
+    """Every exported index set against the oracle's (exact up to the boundary band); returns the
+    per-head selections the output rows are checked against (HeadSelections)."""
     hw = _hw()
-    exact = {}
+    sels = HeadSelections(sel)
     for h, hc in enumerate(heads):
         if hc.kind == PROBE:
             keys = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h)
-            exact[h] = check_probe(keys, case.L, sel, h, hc.k, f"probe head {h}")
+            sels.accept(case.L, h, hc, keys, check_probe(keys, case.L, sel, h, hc.k, f"probe head {h}"))
         elif hc.kind in (CORR, HYBRID):
             ranked = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(case.L.T, hc.k)
-            exact[h] = check_tiles(ranked, sel, hc.k, f"tile head {h}")
-    return exact
+            sels.accept(case.L, h, hc, ranked, check_tiles(ranked, sel, hc.k, f"tile head {h}"))
+    return sels
 
 
-def check_rows(case, heads, sel, out, rows_per_head, exact):
+def check_rows(case, heads, sels, out, rows_per_head):
+    """Output rows of every head against the oracle over that head's (validated) set: no head is
+    skipped, also where a boundary tie made the GPU's set differ from the oracle's."""
     out = out.float().cpu().numpy()
     for h, hc in enumerate(heads):
-        if not exact.get(h, True):
-            continue  # a boundary tie was resolved differently: the set is valid but not unique
         rows = rows_per_head(h)
-        ref = O.sparse_rows(case.L, hc, sel, h, case.Q[h], case.K[h], case.V[h], rows)
+        ref = O.sparse_rows(case.L, hc, sels[h], h, case.Q[h], case.K[h], case.V[h], rows)
         compare_outputs(out[h][rows], ref, f"head {h} ({hc.kind})")
+    sels.report(case.wl.name)
 
 
 @pytest.fixture(scope="module")
@@ -78,8 +81,8 @@ def test_tiny_all_rows(tiny, out_fp32):
     heads = tiny.wl.heads
     att, out = run_gpu(tiny, heads, out_fp32)
     sel = oracle_select(tiny, heads)
-    exact = check_selection(tiny, heads, att, sel)
-    check_rows(tiny, heads, sel, out, lambda h: np.arange(tiny.L.N), exact)
+    sels = check_selection(tiny, heads, att, sel)
+    check_rows(tiny, heads, sels, out, lambda h: np.arange(tiny.L.N))
 
 
 def test_tiny_dense(tiny):
@@ -102,8 +105,8 @@ def test_deterministic(tiny):
     assert torch.equal(a, b)
 
 
-def _custom(S, g, heads, seed=7, M=256, D=128):
-    L = Layout(S=S, g=g, H=len(heads))
+def _custom(S, g, heads, seed=7, M=256, D=128, ns=5):
+    L = Layout(S=S, g=g, H=len(heads), n_special=ns)
     return Workload("custom", L, M=M, delta=11, D=D, heads=heads, seed=seed)
 
 
@@ -139,8 +142,8 @@ def test_edge_cases_all_rows(name):
     heads = case.wl.heads
     att, out = run_gpu(case, heads)
     sel = oracle_select(case, heads)
-    exact = check_selection(case, heads, att, sel)
-    check_rows(case, heads, sel, out, lambda h: np.arange(case.L.N), exact)
+    sels = check_selection(case, heads, att, sel)
+    check_rows(case, heads, sels, out, lambda h: np.arange(case.L.N))
 
 
 def test_cache_mismatch_is_reported_and_out_untouched(tiny):
@@ -169,8 +172,8 @@ def test_s32_selection_and_sampled_rows(s32):
     heads = s32.wl.heads
     att, out = run_gpu(s32, heads, out_fp32=False)
     sel = oracle_select(s32, heads)
-    exact = check_selection(s32, heads, att, sel)
-    check_rows(s32, heads, sel, out, lambda h: sample_rows(s32.wl, h, 512), exact)
+    sels = check_selection(s32, heads, att, sel)
+    check_rows(s32, heads, sels, out, lambda h: sample_rows(s32.wl, h, 512))
 
 
 def test_s32_hybrid_heads_sampled_rows_and_pairs(s32):
@@ -179,12 +182,67 @@ def test_s32_hybrid_heads_sampled_rows_and_pairs(s32):
     heads = [HeadCfg(HYBRID, k=32, stride=20, phase=h % 20) for h in range(s32.L.H)]
     att, out = run_gpu(s32, heads, out_fp32=False)
     sel = oracle_select(s32, heads)
-    exact = check_selection(s32, heads, att, sel)
-    check_rows(s32, heads, sel, out, lambda h: sample_rows(s32.wl, h, 256), exact)
+    sels = check_selection(s32, heads, att, sel)
+    check_rows(s32, heads, sels, out, lambda h: sample_rows(s32.wl, h, 256))
     pairs = hw.saf3r_kept_pairs(att.layout, att.cfg, att.cache)
     for h in (0, 7):
-        if exact.get(h, True):
-            assert int(pairs[h]) == O.kept_pairs(s32.L, heads[h], sel, h)
+        assert int(pairs[h]) == O.kept_pairs(s32.L, heads[h], sels[h], h)
+
+
+# ---------------------------------------------------------------- forced ties of the probe and tile Top-K
+
+@pytest.mark.parametrize("n_rows", [3, 17])
+def test_probe_ties_go_to_the_lower_index(n_rows):
+    """Every patch key of the probe heads takes one of n_rows distinct K rows, so the probe scores
+    tie in groups and the k-th score falls inside a tie group (k = 1 takes one of a group).  Ties
+    go to the lower token index on both sides (section 4.3's Top-K, read with that tie rule), so
+    the sets must be identical, not merely equal up to the boundary band."""
+    case = Case(_custom(4, 12, [HeadCfg(PROBE, k=100), HeadCfg(PROBE, k=37), HeadCfg(PROBE, k=1),
+                                HeadCfg(SCAN, stride=3, phase=1)], seed=70 + n_rows))
+    L = case.L
+    rng = np.random.default_rng(700 + n_rows)
+    patch = O.patch_tokens(L)
+    tmpl = patch[rng.choice(len(patch), size=n_rows, replace=False)]
+    src = np.arange(L.N)
+    src[patch] = tmpl[rng.integers(0, n_rows, size=len(patch))]
+    src_t = torch.from_numpy(src).cuda()
+    for h in range(3):
+        case.k[h] = case.k[h][src_t]
+    case.K = bf16_to_f32(case.k)
+    heads = case.wl.heads
+    att, out = run_gpu(case, heads)
+    sel = oracle_select(case, heads)
+    for h in range(3):  # the ties really are at the boundary
+        sc = sel.probe_scores[h][patch]
+        kth = np.sort(sc)[::-1][heads[h].k - 1]
+        assert np.count_nonzero(sc == kth) > 1
+    sels = check_selection(case, heads, att, sel)
+    assert not sels.over_gpu, f"probe heads {sels.over_gpu} broke a tie differently from the oracle"
+    check_rows(case, heads, sels, out, lambda h: np.arange(L.N))
+
+
+@pytest.mark.parametrize("period", [2, 3])
+def test_tile_ties_go_to_the_lower_index(period):
+    """Views s and s + period get the same DINO features on a layout whose views are exactly two
+    64-token tiles (11x11 patches + 7 special tokens = 128 tokens), so the tiles of those views
+    have identical means and every query tile sees exact cosine ties, its own tile among them.
+    Budgets cut through the tie groups; ties go to the lower tile index on both sides, so the
+    ranked lists of the correspondence and hybrid heads must be identical to the oracle's."""
+    heads = [HeadCfg(CORR, k=2), HeadCfg(CORR, k=4), HeadCfg(HYBRID, k=5, stride=7, phase=2),
+             HeadCfg(HYBRID, k=1, stride=16, phase=0)]
+    case = Case(_custom(6, 11, heads, seed=80 + period, ns=7))
+    L = case.L
+    assert L.V == 128 and L.T == 2 * L.S
+    base = case.dino.cpu().numpy()[:period * L.P].reshape(period, L.P, L.dino_dim)
+    case.dino = torch.from_numpy(np.ascontiguousarray(
+        np.concatenate([base[s % period] for s in range(L.S)], axis=0))).cuda()
+    att, out = run_gpu(case, heads)
+    sel = oracle_select(case, heads)
+    for u in range(L.T):  # each tile's copies tie with it exactly
+        assert np.count_nonzero(sel.tile_cos[u] == sel.tile_cos[u, u]) == L.S // period
+    sels = check_selection(case, heads, att, sel)
+    assert not sels.over_gpu, f"tile heads {sels.over_gpu} broke a tie differently from the oracle"
+    check_rows(case, heads, sels, out, lambda h: np.arange(L.N))
 
 
 # ---------------------------------------------------------------- token-wise per-frame DINO Top-K
@@ -199,7 +257,9 @@ TOKEN_CASES = {
 }
 
 
-def _check_token_heads(case, heads, att, sel, rows):
+def _check_token_heads(case, heads, att, sels, rows):
+    """Per-frame lists of every token-wise head (the given query rows) against the oracle; each
+    head is added to `sels`.  Returns {head: lists identical}."""
     hw = _hw()
     L = case.L
     exact = {}
@@ -207,7 +267,8 @@ def _check_token_heads(case, heads, att, sel, rows):
         if hc.kind != TOKEN:
             continue
         lists = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(L.S * L.P, L.S, hc.k)
-        exact[h] = check_token_lists(lists, L, sel.unit, hc.k, rows, f"token head {h}")
+        exact[h] = check_token_lists(lists, L, sels.base.unit, hc.k, rows(h), f"token head {h}")
+        sels.accept(L, h, hc, lists, exact[h])
     return exact
 
 
@@ -218,13 +279,13 @@ def test_token_heads_all_rows(name):
     heads = case.wl.heads
     att, out = run_gpu(case, heads)
     sel = oracle_select(case, heads)
-    exact = check_selection(case, heads, att, sel)
-    exact.update(_check_token_heads(case, heads, att, sel, np.arange(case.L.N)))
-    check_rows(case, heads, sel, out, lambda h: np.arange(case.L.N), exact)
+    sels = check_selection(case, heads, att, sel)
+    _check_token_heads(case, heads, att, sels, lambda h: np.arange(case.L.N))
+    check_rows(case, heads, sels, out, lambda h: np.arange(case.L.N))
     pairs = hw.saf3r_kept_pairs(att.layout, att.cfg, att.cache)
     for h, hc in enumerate(heads):
         if hc.kind == TOKEN:
-            assert int(pairs[h]) == sum(O.kept_count(case.L, hc, sel, h, i) for i in range(case.L.N))
+            assert int(pairs[h]) == sum(O.kept_count(case.L, hc, sels[h], h, i) for i in range(case.L.N))
 
 
 @pytest.mark.parametrize("n_feat", [2, 5])
@@ -242,10 +303,10 @@ def test_token_heads_tied_features(n_feat):
     heads = case.wl.heads
     att, out = run_gpu(case, heads)
     sel = oracle_select(case, heads)
-    exact = check_selection(case, heads, att, sel)
-    exact.update(_check_token_heads(case, heads, att, sel, np.arange(L.N)))
+    sels = check_selection(case, heads, att, sel)
+    exact = _check_token_heads(case, heads, att, sels, lambda h: np.arange(L.N))
     assert all(exact[h] for h in range(3)), exact
-    check_rows(case, heads, sel, out, lambda h: np.arange(L.N), exact)
+    check_rows(case, heads, sels, out, lambda h: np.arange(L.N))
 
 
 def test_s32_token_heads_sampled_rows(s32):
@@ -253,11 +314,7 @@ def test_s32_token_heads_sampled_rows(s32):
     heads = [HeadCfg(TOKEN, k=16)] * 4 + list(s32.wl.heads[4:])
     att, out = run_gpu(s32, heads, out_fp32=False)
     sel = oracle_select(s32, heads)
-    exact = check_selection(s32, heads, att, sel)
+    sels = check_selection(s32, heads, att, sel)
     rows = {h: sample_rows(s32.wl, h, 64) for h in range(4)}
-    hw = _hw()
-    L = s32.L
-    for h in range(4):
-        lists = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(L.S * L.P, L.S, 16)
-        exact[h] = check_token_lists(lists, L, sel.unit, 16, rows[h], f"token head {h}")
-    check_rows(s32, heads, sel, out, lambda h: rows[h] if h < 4 else sample_rows(s32.wl, h, 128), exact)
+    _check_token_heads(s32, heads, att, sels, lambda h: rows[h])
+    check_rows(s32, heads, sels, out, lambda h: rows[h] if h < 4 else sample_rows(s32.wl, h, 128))

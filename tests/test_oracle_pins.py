@@ -388,3 +388,53 @@ def test_selection_stable_under_fp32_accumulation():
         s_i, loc = O.token_parts(L, i)
         lists[s_i * L.P + loc - L.n_special] = O.token_topk_row(L, s32.unit, i, 12)
     check_token_lists(lists, L, s64.unit, 12, rows, "token fp32")
+
+
+# ---------------------------------------------------------------- row batching of the oracle
+
+@pytest.mark.parametrize("hc", [HeadCfg(POSITION), HeadCfg(POSITION, radius=0), HeadCfg(POSITION, radius=2),
+                                HeadCfg(POSITION, radius=-1), HeadCfg(PROBE, k=30), HeadCfg(CORR, k=2),
+                                HeadCfg(HYBRID, k=2, stride=5, phase=3), HeadCfg(SCAN, stride=4, phase=1),
+                                HeadCfg(DENSE), HeadCfg(TOKEN, k=3)])
+def test_sparse_rows_batching_equals_one_row_at_a_time(hc):
+    """sparse_rows evaluates rows in batches of equal key sets; each output row must equal the
+    plain attention of that row over its own key set, taken one row at a time (rows given in a
+    shuffled order, three views so that rows of the same grid cell and tile sit in different views)."""
+    L = Layout(S=3, g=6, H=1)
+    rng = np.random.default_rng(77)
+    Q, K, V = (rng.standard_normal((1, L.N, 64)) for _ in range(3))
+    dino = rng.standard_normal((L.S * L.P, L.dino_dim)).astype(np.float32)
+    sel = O.select(L, [hc], Q, K, dino)
+    rows = rng.permutation(L.N)
+    got = O.sparse_rows(L, hc, sel, 0, Q[0], K[0], V[0], rows)
+    for n, i in enumerate(rows):
+        keys = O.key_set(L, hc, sel, 0, int(i))
+        want = O.attention_rows(Q[0][i], K[0][keys], V[0][keys])[0]
+        np.testing.assert_allclose(got[n], want, rtol=0, atol=1e-12, err_msg=f"row {i}")
+
+
+def test_given_token_lists_replace_the_ranking():
+    """A token-wise head evaluated over given per-frame lists: the oracle's own lists give the
+    same sets as its ranking, and a list that swaps one key changes exactly that row's set."""
+    L = Layout(S=3, g=5, H=1)
+    rng = np.random.default_rng(78)
+    dino = rng.standard_normal((L.S * L.P, L.dino_dim)).astype(np.float32)
+    hc = HeadCfg(TOKEN, k=2)
+    sel = O.select(L, [hc], None, None, dino)
+    lists = np.stack([O.token_topk_row(L, sel.unit, L.n_special + p % L.P + (p // L.P) * L.V, 2)
+                      for p in range(L.S * L.P)])
+    given = O.Selection()
+    given.unit = sel.unit
+    given.token_lists = {0: lists}
+    for i in range(L.N):
+        assert np.array_equal(O.key_set(L, hc, sel, 0, i), O.key_set(L, hc, given, 0, i))
+    swapped = lists.copy()
+    i = 2 * L.V + L.n_special + 7  # view 2, patch 7
+    a = 2 * L.P + 7
+    old = swapped[a, 1, 1]
+    new = next(p for p in range(L.P) if p not in swapped[a, 1])
+    swapped[a, 1, 1] = new
+    given.token_lists = {0: swapped}
+    diff = set(O.key_set(L, hc, sel, 0, i).tolist()) ^ set(O.key_set(L, hc, given, 0, i).tolist())
+    assert diff == {1 * L.V + L.n_special + old, 1 * L.V + L.n_special + new}
+    assert np.array_equal(O.key_set(L, hc, sel, 0, i + 1), O.key_set(L, hc, given, 0, i + 1))
