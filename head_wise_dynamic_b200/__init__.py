@@ -9,7 +9,6 @@ the compiled library and a B200.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 from dataclasses import dataclass
 from typing import List, Optional, Sequence
@@ -83,6 +82,12 @@ def lib() -> ctypes.CDLL:
         L.saf3r_choose_eq2.restype = i32
         L.saf3r_set_kernel_events.argtypes = [vp, vp]
         L.saf3r_set_kernel_events.restype = None
+        L.saf3r_set_wait_budget.argtypes = [ctypes.c_longlong]
+        L.saf3r_set_wait_budget.restype = None
+        L.saf3r_test_withhold_arrive.argtypes = []
+        L.saf3r_test_withhold_arrive.restype = None
+        L.saf3r_baseline_stride.argtypes = [ctypes.c_double]
+        L.saf3r_baseline_stride.restype = ctypes.c_int32
         L.saf3r_check.argtypes = [vp]
         L.saf3r_check.restype = i32
         L.saf3r_last_launch_count.argtypes = []
@@ -240,11 +245,15 @@ def saf3r_choose_eq2(nmse, pairs, base: int):
     return choice, mean
 
 
-def baseline_stride(sigma: float) -> int:
-    """Stride of the uniform-sampling baseline of sparsity at least sigma: ceil(1 / (1 - sigma))."""
-    if not 0.0 <= sigma < 1.0:
+def saf3r_baseline_stride(sigma: float) -> int:
+    """Stride of the uniform-sampling baseline of sparsity at least sigma (the library's rule)."""
+    s = int(lib().saf3r_baseline_stride(float(sigma)))
+    if s < 1:
         raise ValueError("sigma must be in [0, 1)")
-    return int(math.ceil(1.0 / (1.0 - sigma) - 1e-9))
+    return s
+
+
+baseline_stride = saf3r_baseline_stride
 
 
 def profile_heads_eq2(layout, cand, base: int, inputs, workspace, stream=None):
@@ -292,6 +301,16 @@ def saf3r_set_kernel_events(start=None, stop=None):
     torch creates CUDA events lazily: record each event once before handing it over."""
     lib().saf3r_set_kernel_events(None if start is None else start.cuda_event,
                                   None if stop is None else stop.cuda_event)
+
+
+def saf3r_set_wait_budget(cycles: int = 0):
+    """Budget (GPU clock cycles) of every bounded device wait of this thread's following calls; 0 = default."""
+    lib().saf3r_set_wait_budget(int(cycles))
+
+
+def saf3r_test_withhold_arrive():
+    """Test hook: the next attention launch on this thread lets one pipeline wait run out (see saf3r.h)."""
+    lib().saf3r_test_withhold_arrive()
 
 
 def saf3r_check(stream=None):

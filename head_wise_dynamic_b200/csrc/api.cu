@@ -23,7 +23,9 @@ __device__ int g_device_error;  // the one piece of library state: first device-
 thread_local int t_launches = 0;
 thread_local cudaEvent_t t_ev_start = nullptr, t_ev_stop = nullptr;
 
-constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (~2 s) before a device wait gives up
+constexpr long long kWaitBudget = 4000000000LL;  // default: clock cycles (~2 s) before a device wait gives up
+thread_local long long t_wait_budget = kWaitBudget;
+thread_local bool t_withhold_arrive = false;       // test hook, consumed by the next attention launch
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -485,7 +487,9 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   p.T = d.T;
   p.err = dev.err;
   p.ok_flag = ok_flag;
-  p.wait_budget = kWaitBudget;
+  p.wait_budget = t_wait_budget;
+  p.withhold_arrive = t_withhold_arrive ? 1 : 0;
+  t_withhold_arrive = false;
 
   if (t_ev_start && t_ev_stop && cudaEventRecord(t_ev_start, stream) != cudaSuccess) return SAF3R_ERR_CUDA;
   if (n_main > 0) {
@@ -526,6 +530,12 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
 
 }  // namespace
 
+saf3r_status saf3r::validate_layout_cfg(const saf3r_layout* L, const saf3r_head_cfg* cfg) {
+  const saf3r_status st = check_layout(L);
+  if (st != SAF3R_OK) return st;
+  return check_cfg(make_dims(*L), cfg, L->H);
+}
+
 bool saf3r::make_map_f16_rows(CUtensorMap* m, const void* base, long long rows, int cols) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
@@ -558,6 +568,18 @@ int saf3r_last_launch_count(void) { return t_launches; }
 void saf3r_set_kernel_events(void* start, void* stop) {
   t_ev_start = static_cast<cudaEvent_t>(start);
   t_ev_stop = static_cast<cudaEvent_t>(stop);
+}
+
+void saf3r_set_wait_budget(long long cycles) { t_wait_budget = cycles > 0 ? cycles : kWaitBudget; }
+
+void saf3r_test_withhold_arrive(void) { t_withhold_arrive = true; }
+
+int32_t saf3r_baseline_stride(double sigma) {
+  if (!(sigma >= 0.0 && sigma < 1.0)) return -1;
+  // the smallest s with sparsity 1 - 1/s >= sigma (the 1e-12 absorbs the rounding of 1 - 1/s)
+  int32_t s = 1;
+  while (1.0 - 1.0 / s < sigma - 1e-12) ++s;
+  return s;
 }
 
 size_t saf3r_cache_bytes(const saf3r_layout* L, const saf3r_head_cfg* cfg) {
@@ -620,7 +642,7 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   sp.tok_off = cl.tok_off;
   sp.num_sms = dev.sms;
   sp.err = dev.err;
-  sp.wait_budget = kWaitBudget;
+  sp.wait_budget = t_wait_budget;
   CacheHeader& hd = sp.header;
   std::memset(&hd, 0, sizeof(hd));
   hd.magic = kCacheMagic;
@@ -846,7 +868,7 @@ saf3r_status saf3r_profile_heads(const saf3r_layout* L, const saf3r_head_cfg* ca
   for (int c = 0; c < n_cand; ++c) {
     for (int h = 0; h < d.H; ++h) cfg[h] = apply_candidate(cand[c], h);
     if ((st = check_cfg(d, cfg.data(), d.H)) != SAF3R_OK) return st;
-    any_corr |= tile_kind(cand[c].type);
+    any_corr |= tile_kind(cand[c].type) || cand[c].type == SAF3R_TOKEN;
   }
   if (any_corr && !dino) return SAF3R_ERR_INVALID;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

@@ -226,7 +226,7 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm,
   }
   // Teardown: every copy this thread issued must have landed before the CTA exits
   // (these waits ignore the abort flag but stay bounded).
-  const long long drain = budget / 4;
+  const long long drain = kDrainBudget;
   if (q_issued > 0) mbar_wait_drain(&sm.q_full, (q_issued - 1) & 1, drain);
   for (uint32_t c = (k_issued > kStages ? k_issued - kStages : 0); c < k_issued; ++c)
     mbar_wait_drain(&sm.k_full[c % kStages], (c / kStages) & 1, drain);
@@ -375,6 +375,7 @@ struct RowCtx {
   uint32_t lane_off; // TMEM lane field of this warp
   int nb_lo[2][kNbIntervals], nb_hi[2][kNbIntervals];  // position heads: kept derived rows [lo, hi) per tile
   int lat_stride, lat_phase;  // hybrid heads: the lattice (counted in the derived run), 0 = none
+  bool withhold;     // test hook: skip the next P-ready arrival (the MMA warp's wait then runs out)
 };
 
 // Bits b of a 64-key half-block starting at token j0 whose token j0 + b lies on the lattice
@@ -408,6 +409,15 @@ __device__ __forceinline__ uint64_t key_mask(const Half& hb, const RowCtx& rc, i
     v &= nb;
   }
   return v;
+}
+
+// This warp's share of "P_t is in TMEM" (p_full counts one arrival per softmax warp).
+__device__ __forceinline__ void arrive_p_full(AttnSmem& sm, RowCtx& rc, int t) {
+  if (rc.withhold) {  // test hook only: this one arrival never comes
+    rc.withhold = false;
+    return;
+  }
+  if (rc.lane == 0) mbar_arrive(&sm.p_full[t]);
 }
 
 struct SoftmaxState {
@@ -453,7 +463,7 @@ __device__ __forceinline__ void exponentials(const float (&s)[64], float m, uint
 // P (bf16) written over the half's first 32 S columns, arrival on p_full[t].
 template <int kMask>
 __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, SoftmaxState& ss, uint32_t tmem,
-                                             const RowCtx& rc, int t, int j, uint64_t valid, float& m, float& l) {
+                                             RowCtx& rc, int t, int j, uint64_t valid, float& m, float& l) {
   if (!__all_sync(0xffffffffu,
                   mbar_wait(&sm.s_full[t], ss.sfull_c[t] & 1, &sm.abort, p.err, p.wait_budget, SAF3R_ERR_TIMEOUT)))
     return false;
@@ -470,7 +480,7 @@ __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, 
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (rc.lane == 0) mbar_arrive(&sm.p_full[t]);
+    arrive_p_full(sm, rc, t);
     return true;
   }
   float s[64];
@@ -551,14 +561,14 @@ __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, 
   tmem_wait_st();
   tc_fence_before();
   __syncwarp();
-  if (rc.lane == 0) mbar_arrive(&sm.p_full[t]);
+  arrive_p_full(sm, rc, t);
   return true;
 }
 
 // All key blocks of one item: tile 0 then tile 1 for every block.
 template <int kMask>
 __device__ __forceinline__ bool softmax_blocks(const AttnParams& p, AttnSmem& sm, SoftmaxState& ss, uint32_t tmem,
-                                               ItemInfo& it, const RowCtx& rc, float (&m)[2], float (&l)[2]) {
+                                               ItemInfo& it, RowCtx& rc, float (&m)[2], float (&l)[2]) {
   for (int j = 0; j < it.nblk; ++j) {
     Half hb;
     if (kMask == kMaskPlain) {
@@ -595,6 +605,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
   rc.r = wq * 32 + lane;
   rc.lane = lane;
   rc.lane_off = static_cast<uint32_t>(wq * 32) << 16;
+  rc.withhold = p.withhold_arrive != 0 && blockIdx.x == 0 && warp == 4;
   const int r = rc.r;
   SoftmaxState ss;
   bool ok = true;

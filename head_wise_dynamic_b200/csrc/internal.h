@@ -13,6 +13,9 @@ constexpr int kItemRows = 256;    // query rows of one attention work item (two 
 constexpr int kMaxRadius = 3;
 constexpr int kTokenMaxDim = 384;  // DINO width the token-wise selection keeps in registers
 constexpr uint32_t kCacheMagic = 0x52334653u;  // "SF3R"
+// Teardown waits (copies already issued must land before a CTA exits) have their own fixed
+// budget, independent of the per-call wait budget, so a short test budget cannot cut them off.
+constexpr long long kDrainBudget = 1000000000LL;  // clock cycles (~0.5 s)
 constexpr uint32_t kCacheVersion = 2;
 
 // Heads whose keys include ranked DINO tiles (they share the cached tile lists), and heads
@@ -98,6 +101,7 @@ struct AttnParams {
   int* err;
   const int* ok_flag;  // nonzero: cache check passed (NULL: no check)
   long long wait_budget;
+  int32_t withhold_arrive;  // test hook: CTA 0's first softmax warp withholds its first P-ready arrival
   HeadPlan heads[kMaxHeads];
 };
 
@@ -175,6 +179,9 @@ struct DerivedArgs {
 #include <cuda_runtime.h>
 
 namespace saf3r {
+
+// check_layout + check_cfg of the C ABI (api.cu): SAF3R_OK, SAF3R_ERR_INVALID or SAF3R_ERR_UNSUPPORTED
+saf3r_status validate_layout_cfg(const saf3r_layout* L, const saf3r_head_cfg* cfg);
 
 // launchers (each returns the launch error, if any)
 size_t attn_smem_bytes();

@@ -52,6 +52,8 @@ saf3r_status scratch_address(void** out) {
 extern "C" saf3r_status saf3r_select_kv_static(const saf3r_layout* layout, const saf3r_head_cfg* cfg,
                                                const void* q, const void* k, const float* dino, void* cache,
                                                void* stream) {
+  const saf3r_status valid = saf3r::validate_layout_cfg(layout, cfg);  // the codes saf3r_select_kv returns
+  if (valid != SAF3R_OK) return valid;
   const size_t need = saf3r_workspace_bytes(layout, cfg, SAF3R_OP_SELECT);
   if (need == 0) return SAF3R_ERR_INVALID;
   if (need > kStaticScratchBytes) return SAF3R_ERR_UNSUPPORTED;  // layer too large for the built-in scratch

@@ -93,7 +93,7 @@ __device__ void sim_producer(const TokenSimParams& p, SimSmem& sm, const CUtenso
     }
   }
   // every copy issued must land before the CTA exits (bounded, ignores the abort flag)
-  const long long drain = p.wait_budget / 4;
+  const long long drain = kDrainBudget;
   for (uint32_t c = (it > kSimStages ? it - kSimStages : 0); c < it; ++c)
     mbar_wait_drain(&sm.full[c % kSimStages], (c / kSimStages) & 1, drain);
 }
@@ -139,7 +139,7 @@ __device__ void sim_mma(const TokenSimParams& p, SimSmem& sm, uint32_t tmem) {
   if (issued) {
     if (elect_one()) mma_commit(&sm.drained);
     __syncwarp();
-    mbar_wait_drain(&sm.drained, 0, p.wait_budget / 4);
+    mbar_wait_drain(&sm.drained, 0, kDrainBudget);
   }
 }
 

@@ -229,6 +229,15 @@ saf3r_status saf3r_choose_eq2(int n_inputs, int H, int n_cand, const double* nms
                               int base, int32_t* choice, double* nmse_mean);
 
 /*
+ * Stride of the uniform-sampling baseline from which the eq. 2 search starts
+ * (section 4.2: uniform sampling at sparsity ratio sigma; section 5.1 uses
+ * sigma = 0.85): keeping one key in s has sparsity 1 - 1/s, so the baseline
+ * stride is the smallest s with 1 - 1/s >= sigma, i.e. ceil(1 / (1 - sigma))
+ * (7 for sigma = 0.85).  Returns -1 for sigma outside [0, 1).  Host only.
+ */
+int32_t saf3r_baseline_stride(double sigma);
+
+/*
  * Copy one head's cached index list to host memory (synchronizes `stream`):
  * PROBE head -> its k kept patch keys (ascending); CORR or HYBRID head -> the
  * ranked tile list int32 [T][k] truncated to that head's k; TOKEN head -> the
@@ -256,6 +265,28 @@ saf3r_status saf3r_kept_pairs(const saf3r_layout* layout, const saf3r_head_cfg* 
  * hook off.  The events are owned by the caller.
  */
 void saf3r_set_kernel_events(void* start, void* stop);
+
+/*
+ * Budget, in GPU clock cycles, of every bounded device wait (the attention
+ * kernel's and the token-wise selection's pipeline waits) in the calls that
+ * follow on this host thread; cycles <= 0 restores the default of 4e9 cycles
+ * (about 2 s at 1.965 GHz).  When a wait runs out, its CTA records
+ * SAF3R_ERR_TIMEOUT in the device error word, lets the copies it has in flight
+ * land (a separate, fixed teardown budget), frees its tensor memory and exits;
+ * the output rows of its unfinished work items are then left unwritten.
+ */
+void saf3r_set_wait_budget(long long cycles);
+
+/*
+ * Test hook for the timeout path.  The next saf3r_sparse_attn or
+ * saf3r_dense_attn call on this host thread launches its attention kernel with
+ * one softmax warp of the first CTA withholding its first "P is in tensor
+ * memory" arrival, so the tensor-core warp's wait for it runs out after the wait
+ * budget (see saf3r_set_wait_budget): nothing faults or hangs, every device wait
+ * being bounded.  saf3r_check then returns SAF3R_ERR_TIMEOUT; the following
+ * calls run normally.  Not for production use.
+ */
+void saf3r_test_withhold_arrive(void);
 
 /*
  * Synchronize `stream`, then read and clear the calling device's error word.

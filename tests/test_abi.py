@@ -132,3 +132,43 @@ def test_token_select_workspace_on_host(S):
     chunk = min(R, max(128, (1 << 30) // (2 * ld) // 128 * 128))
     assert w1 - w0 >= feats + chunk * ld * 2
     assert w1 - w0 <= feats + min(R * ld * 2, (1 << 30)) + 4096
+
+
+def test_baseline_stride_rule_in_the_library():
+    import oracle as O
+    for sigma in (0.0, 0.5, 0.75, 0.8, 0.85, 0.875, 0.9, 0.95, 0.96875, 0.99):
+        assert hw.saf3r_baseline_stride(sigma) == O.baseline_stride(sigma), sigma
+    assert hw.saf3r_baseline_stride(0.85) == 7  # section 5.1's sigma
+    for bad in (-0.1, 1.0, 1.5, float("nan")):
+        assert hw.lib().saf3r_baseline_stride(bad) == -1
+
+
+def test_static_select_returns_the_regular_entry_points_codes():
+    """saf3r_select_kv_static validates like saf3r_select_kv (before any device work)."""
+    L, cfg = _tiny()
+    f = hw.lib().saf3r_select_kv_static
+    f.argtypes = [ctypes.POINTER(hw.saf3r_layout), ctypes.POINTER(hw.saf3r_head_cfg)] + [ctypes.c_void_p] * 5
+    f.restype = ctypes.c_int
+    p = 0x1000
+    L.d = 128
+    assert f(ctypes.byref(L), cfg, p, p, p, p, None) == hw.ERR_UNSUPPORTED
+    L, cfg = _tiny()
+    cfg[1].k = 0
+    assert f(ctypes.byref(L), cfg, p, p, p, p, None) == hw.ERR_INVALID
+    L, cfg = _tiny()
+    L.dino_dim = 512
+    tok = hw.cfg_array([HeadCfg(TOKEN, k=4)] + list(WORKLOADS["tiny"].heads[1:]))
+    assert f(ctypes.byref(L), tok, p, p, p, p, None) == hw.ERR_UNSUPPORTED
+
+
+def test_profile_rejects_a_token_candidate_without_dino():
+    L, _ = _tiny()
+    cand = hw.cfg_array([HeadCfg(TOKEN, k=4), HeadCfg(SCAN, stride=4)])
+    lib = hw.lib()
+    H = L.H
+    chosen = (hw.saf3r_head_cfg * H)()
+    nmse = (ctypes.c_double * (H * 2))()
+    pairs = (ctypes.c_int64 * (H * 2))()
+    p = 0x1000
+    assert lib.saf3r_profile_heads(ctypes.byref(L), cand, 2, p, p, p, None, 0.01, chosen, nmse, pairs, p,
+                                   None) == hw.ERR_INVALID
