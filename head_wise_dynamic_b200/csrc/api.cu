@@ -259,6 +259,12 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
       case SAF3R_PROBE:
         rows = nsp + c.k;
         break;
+      case SAF3R_TOKEN:  // the special-token queries, gathered for the tensor-core kernel
+        if (nsp > 0) {
+          s.qc_begin[h] = static_cast<int>(s.qc_rows);
+          s.qc_rows += nsp;
+        }
+        break;
       case SAF3R_SCAN:
       case SAF3R_HYBRID: {  // the lattice, then the specials off it
         s.n_lat[h] = (d.N - c.phase + c.stride - 1) / c.stride;
@@ -423,7 +429,8 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   // attention
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
-  // token-wise heads run in their own kernel (no shared key runs); the others in the MMA kernel
+  // the patch queries of token-wise heads run in their own kernel (no shared key runs); their
+  // special-token queries (every key: dense rows) and every other head in the MMA kernel
   std::vector<int> order;
   TokenAttnParams tp;
   std::memset(&tp, 0, sizeof(tp));
@@ -432,6 +439,7 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
       tp.heads[tp.n_heads] = h;
       tp.k[tp.n_heads] = cfg[h].k;
       ++tp.n_heads;
+      if (s.qc_begin[h] >= 0) order.push_back(h);
     } else {
       order.push_back(h);
     }
@@ -446,12 +454,12 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     HeadPlan& hp = p.heads[i];
     hp.head = h;
     hp.kind = c.type;
-    hp.q_src = c.type == SAF3R_POSITION ? 1 : (tile_kind(c.type) ? 2 : 0);
+    hp.q_src = c.type == SAF3R_POSITION ? 1 : (tile_kind(c.type) ? 2 : (c.type == SAF3R_TOKEN ? 3 : 0));
     hp.q_base = tile_kind(c.type) ? cl.order_off : (s.qc_begin[h] < 0 ? 0 : s.qc_begin[h]);
     hp.lat_stride = c.type == SAF3R_HYBRID ? c.stride : 0;
     hp.lat_phase = c.type == SAF3R_HYBRID ? c.phase : 0;
     hp.kc_base = s.kc_begin[h];
-    hp.n_items = items_of(d.N);
+    hp.n_items = c.type == SAF3R_TOKEN ? items_of(d.ns * d.S) : items_of(d.N);
     hp.item_begin = item;
     item += hp.n_items;
     hp.seg_list = -1;
@@ -465,6 +473,7 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
         hp.seg = Seg{1, 0, s.n_rows[h], kSegAllQuarters};
         break;
       case SAF3R_DENSE:
+      case SAF3R_TOKEN:  // special-token queries of a token-wise head keep every key
         hp.seg = Seg{0, 0, d.N, kSegAllQuarters};
         break;
       default: {

@@ -32,6 +32,13 @@
 // which walks the list anyway, leaves each block's halves in shared memory next to its V
 // stage.  Warps whose 32 rows keep no key of a half-block (correspondence tiles of another
 // quarter, cells outside the neighbourhood) write P = 0 without computing anything.
+//
+// Exponentials: one pair in eight (kPolyPairs) is computed on the FMA pipe instead of the SFU,
+// which the softmax otherwise keeps busiest: 2^x = 2^floor(x) * p(x - floor(x)), the floor from
+// one round-down addition of 1.5 * 2^23, p a cubic fitted to 2^f on [0, 1) for least maximum
+// relative error (a linear-programming minimax fit with p(0) = 1: relative error below 8.6e-5,
+// far below the 2^-9 of the bf16 P it feeds), and 2^floor(x) added to p's exponent field.  x is
+// clamped at -127 first, where the construction gives exactly +0 (masked keys).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -50,6 +57,13 @@ constexpr int kTileBytes = 128 * 64 * 2;  // 128 rows x 64 bf16
 constexpr int kHalfBytes = 64 * 64 * 2;   // 64 rows x 64 bf16
 constexpr float kScaleLog2 = 0.18033688011112042f;  // log2(e) / sqrt(64)
 constexpr float kRescaleThreshold = 8.0f;           // log2 units: keep a stale max until it is 256x off
+// Pairs (of the 32 per 64-key half-block) whose exponentials run on the FMA pipe: bit i = pair i.
+#ifndef SAF3R_POLY_PAIRS
+#define SAF3R_POLY_PAIRS 0x80808080u
+#endif
+constexpr uint32_t kPolyPairs = SAF3R_POLY_PAIRS;
+// the cubic of the FMA-pipe exponential: p(f) = 1 + f (c1 + f (c2 + f c3))
+constexpr float kExpC1 = 0.6951168179512024f, kExpC2 = 0.22764486074447632f, kExpC3 = 0.07706713676452637f;
 
 // One 64-row half-block of keys.
 struct Half {
@@ -187,7 +201,7 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm,
     mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
     for (int quarter = 0; quarter < 4; ++quarter) {
       void* dst = sm.q[quarter >> 1] + (quarter & 1) * kHalfBytes;
-      if (hp.q_src == 1) {
+      if (hp.q_src == 1 || hp.q_src == 3) {
         tma_load_2d(dst, &tmQC, 0, hp.q_base + it.q0 + quarter * 64, &sm.q_full);
       } else {
         int row = it.q0 + quarter * 64;
@@ -443,19 +457,52 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
   }
 }
 
+// 2^x0, 2^x1 on the FMA pipe (see the head of this file).
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float& e1) {
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23: x + kMagic rounded down holds floor(x) in its low bits
+  x0 = fmaxf(x0, -127.f);
+  x1 = fmaxf(x1, -127.f);
+  uint64_t t, xi, f, pp;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(t) : "l"(f32x2(x0, x1)), "l"(f32x2(kMagic, kMagic)));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(xi) : "l"(t), "l"(f32x2(kMagic, kMagic)));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(f32x2(x0, x1)), "l"(xi));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pp) : "l"(f), "l"(f32x2(kExpC3, kExpC3)), "l"(f32x2(kExpC2, kExpC2)));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pp) : "l"(pp), "l"(f), "l"(f32x2(kExpC1, kExpC1)));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pp) : "l"(pp), "l"(f), "l"(f32x2(1.f, 1.f)));
+  // exponent field += floor(x): (bits of t) << 23 is floor(x) << 23 modulo 2^32
+  e0 = __uint_as_float(static_cast<uint32_t>(pp) + (static_cast<uint32_t>(t) << 23));
+  e1 = __uint_as_float(static_cast<uint32_t>(pp >> 32) + (static_cast<uint32_t>(t >> 32) << 23));
+}
+
+// 2^x0, 2^x1 of pair i of a half-block: on the FMA pipe for the pairs of kPolyPairs, else the SFU.
+__device__ __forceinline__ void exp2_pair(int i, float x0, float x1, float& e0, float& e1) {
+  if ((kPolyPairs >> i) & 1u) {
+    exp2_poly2(x0, x1, e0, e1);
+  } else {
+    e0 = fast_exp2(x0);
+    e1 = fast_exp2(x1);
+  }
+}
+
 // P = 2^(s * scale - m) for the row's 64 logits as 32 bf16 pairs, and 8 partial row sums (a
 // single running sum would be a chain of dependent adds).
 __device__ __forceinline__ void exponentials(const float (&s)[64], float m, uint32_t (&pk)[32], float (&rp)[8]) {
   const float m_use = (m == -INFINITY) ? 0.f : m;
 #pragma unroll
   for (int i = 0; i < 8; ++i) rp[i] = 0.f;
+  float x[64];
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    float x0 = s[2 * i], x1 = s[2 * i + 1];
-    ffma2(x0, x1, kScaleLog2, -m_use);
-    const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-    fadd2(rp[2 * (i & 3)], rp[2 * (i & 3) + 1], e0, e1);
-    pk[i] = pack_bf16x2(e0, e1);
+    x[2 * i] = s[2 * i];
+    x[2 * i + 1] = s[2 * i + 1];
+    ffma2(x[2 * i], x[2 * i + 1], kScaleLog2, -m_use);
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) exp2_pair(i, x[2 * i], x[2 * i + 1], x[2 * i], x[2 * i + 1]);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    fadd2(rp[2 * (i & 3)], rp[2 * (i & 3) + 1], x[2 * i], x[2 * i + 1]);
+    pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
   }
 }
 
@@ -513,14 +560,20 @@ __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, 
       rp[i] = 0.f;
       mp[i] = s[i];
     }
+    float x[64];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      float x0 = s[2 * i], x1 = s[2 * i + 1];
-      if (i >= 4) mp[i & 7] = max3f(mp[i & 7], x0, x1);
-      ffma2(x0, x1, kScaleLog2, -m_spec);
-      const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-      fadd2(rp[2 * (i & 3)], rp[2 * (i & 3) + 1], e0, e1);
-      pk[i] = pack_bf16x2(e0, e1);
+      x[2 * i] = s[2 * i];
+      x[2 * i + 1] = s[2 * i + 1];
+      if (i >= 4) mp[i & 7] = max3f(mp[i & 7], x[2 * i], x[2 * i + 1]);
+      ffma2(x[2 * i], x[2 * i + 1], kScaleLog2, -m_spec);
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) exp2_pair(i, x[2 * i], x[2 * i + 1], x[2 * i], x[2 * i + 1]);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      fadd2(rp[2 * (i & 3)], rp[2 * (i & 3) + 1], x[2 * i], x[2 * i + 1]);
+      pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
     }
     const float mx =
         max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * kScaleLog2;
@@ -696,6 +749,8 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
     int token = -1;
     if (hp.q_src == 1) {
       if (qrow < p.N) token = position_token(p, qrow);
+    } else if (hp.q_src == 3) {
+      if (qrow < p.ns * p.S) token = position_token(p, p.P * p.S + qrow);  // the special tokens, view by view
     } else if (hp.q_src == 2) {
       const int u = mapped_tile(p, hp, it.local, quarter);
       if (u >= 0 && u * 64 + (r & 63) < p.N) token = u * 64 + (r & 63);

@@ -12,6 +12,7 @@ constexpr int kMaxHeads = 64;
 constexpr int kItemRows = 256;    // query rows of one attention work item (two 128-row MMA tiles)
 constexpr int kMaxRadius = 3;
 constexpr int kTokenMaxDim = 384;  // DINO width the token-wise selection keeps in registers
+
 constexpr uint32_t kCacheMagic = 0x52334653u;  // "SF3R"
 // Teardown waits (copies already issued must land before a CTA exits) have their own fixed
 // budget, independent of the per-call wait budget, so a short test budget cannot cut them off.
@@ -73,7 +74,8 @@ struct HeadPlan {
   int32_t head;       // head index h in [0, H)
   int32_t kind;       // saf3r_head_type
   int32_t q_src;      // 0: caller Q rows are tokens; 1: derived cell-major Q rows (position heads);
-                      // 2: caller Q, each 64-row quarter of an item is the query tile qmap[4*item + quarter]
+                      // 2: caller Q, each 64-row quarter of an item is the query tile qmap[4*item + quarter];
+                      // 3: derived Q rows of the special tokens only, view by view (token-wise heads)
   int32_t q_base;     // derived Q row base (q_src == 1); qmap offset (q_src == 2)
   int32_t kc_base;    // derived K/V row base
   int32_t n_items;    // work items (256 query rows each)
@@ -106,7 +108,8 @@ struct AttnParams {
 };
 
 
-// Token-wise correspondence heads (token_attn.cu): every query row has its own kept keys.
+// Token-wise correspondence heads (token_attn.cu): every patch query row has its own kept keys
+// (the special-token rows, which keep every key, run in the tensor-core kernel as dense rows).
 struct TokenAttnParams {
   int32_t n_heads;
   int32_t heads[kMaxHeads];   // head index h
@@ -159,7 +162,7 @@ struct DerivedHead {
   int kind;
   int kc_begin;     // first global derived K/V row
   int n_rows;       // derived K/V rows of this head
-  int qc_begin;     // first global derived Q row (position heads), -1 if none
+  int qc_begin;     // first global derived Q row (position and token-wise heads), -1 if none
   int stride, phase, n_lat;  // scan heads
   int probe_off;    // cache int32 offset of the probe key list
   int off_list;     // scan heads: int offset of the off-lattice special list in the workspace

@@ -123,11 +123,15 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(DerivedArgs a, const u
     } else {
       const int row = static_cast<int>(task - a.kc_total);
       int hi = -1;
-      for (int i = 0; i < a.n; ++i)
-        if (a.h[i].qc_begin >= 0 && row >= a.h[i].qc_begin && row < a.h[i].qc_begin + a.N) hi = i;
+      for (int i = 0; i < a.n; ++i) {
+        const int n_q = a.h[i].kind == SAF3R_TOKEN ? a.ns * a.S : a.N;
+        if (a.h[i].qc_begin >= 0 && row >= a.h[i].qc_begin && row < a.h[i].qc_begin + n_q) hi = i;
+      }
       if (hi < 0) continue;
       const DerivedHead& d = a.h[hi];
-      const int tok = cm_query_token(row - d.qc_begin, a.S, a.V, a.ns, a.P);
+      // position heads: every query in cell-major order; token-wise heads: the special tokens
+      const int tok = d.kind == SAF3R_TOKEN ? special_token(row - d.qc_begin, a.V, a.ns)
+                                             : cm_query_token(row - d.qc_begin, a.S, a.V, a.ns, a.P);
       const size_t src = (static_cast<size_t>(d.head) * a.N + tok) * kD;
       reinterpret_cast<uint4*>(qc + static_cast<size_t>(row) * kD)[sub] =
           reinterpret_cast<const uint4*>(q + src)[sub];

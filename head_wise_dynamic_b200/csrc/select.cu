@@ -38,7 +38,34 @@ struct ProbeArgs {
   int cache_off[kMaxHeads];  // int32 offset of the key list in the cache
 };
 
-// Partial fp64 column sums of Q_h over a range of rows.
+// The 8 bf16 features of a 16-byte chunk as fp64, in order.
+__device__ __forceinline__ void bf16x8_to_f64(const uint4& w, double (&x)[8]) {
+  x[0] = static_cast<double>(bf16_lo(w.x));
+  x[1] = static_cast<double>(bf16_hi(w.x));
+  x[2] = static_cast<double>(bf16_lo(w.y));
+  x[3] = static_cast<double>(bf16_hi(w.y));
+  x[4] = static_cast<double>(bf16_lo(w.z));
+  x[5] = static_cast<double>(bf16_hi(w.z));
+  x[6] = static_cast<double>(bf16_lo(w.w));
+  x[7] = static_cast<double>(bf16_hi(w.w));
+}
+
+// acc[i] += feature i of a 16-byte chunk of 8 bf16 features (fp64 sums).
+__device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4& w) {
+  acc[0] += static_cast<double>(bf16_lo(w.x));
+  acc[1] += static_cast<double>(bf16_hi(w.x));
+  acc[2] += static_cast<double>(bf16_lo(w.y));
+  acc[3] += static_cast<double>(bf16_hi(w.y));
+  acc[4] += static_cast<double>(bf16_lo(w.z));
+  acc[5] += static_cast<double>(bf16_hi(w.z));
+  acc[6] += static_cast<double>(bf16_lo(w.w));
+  acc[7] += static_cast<double>(bf16_hi(w.w));
+}
+
+// Partial fp64 column sums of Q_h over a range of rows.  Lane l of a warp reads the 16-byte
+// chunk (l % 8) of row r + l / 8 (a warp reads 4 whole rows, 512 contiguous bytes, per load) and
+// keeps the 8 column sums of its chunk; two rows per lane are in flight per step.  The lanes and
+// warps that share a chunk are added in a fixed order at the end.
 __global__ void __launch_bounds__(256) probe_partial_kernel(const uint16_t* __restrict__ q, int N,
                                                             ProbeArgs a, double* __restrict__ partial) {
   const int hp = blockIdx.y;
@@ -46,53 +73,91 @@ __global__ void __launch_bounds__(256) probe_partial_kernel(const uint16_t* __re
   const int rows_per = (N + gridDim.x - 1) / gridDim.x;
   const int r0 = blockIdx.x * rows_per;
   const int r1 = min(N, r0 + rows_per);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t* qh = reinterpret_cast<const uint32_t*>(q + static_cast<size_t>(h) * N * kD);
-  double s0 = 0.0, s1 = 0.0;
-  for (int r = r0 + warp; r < r1; r += 8) {
-    const uint32_t w = qh[static_cast<size_t>(r) * (kD / 2) + lane];
-    s0 += static_cast<double>(bf16_lo(w));
-    s1 += static_cast<double>(bf16_hi(w));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = lane & 7;
+  const uint4* qh = reinterpret_cast<const uint4*>(q + static_cast<size_t>(h) * N * kD);
+  double acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  int r = r0 + warp * 4 + (lane >> 3);
+  for (; r + 32 < r1; r += 64) {
+    const uint4 w0 = qh[static_cast<size_t>(r) * 8 + sub];
+    const uint4 w1 = qh[static_cast<size_t>(r + 32) * 8 + sub];
+    add_bf16x8(acc, w0);
+    add_bf16x8(acc, w1);
   }
-  __shared__ double acc[8][kD];
-  acc[warp][2 * lane] = s0;
-  acc[warp][2 * lane + 1] = s1;
+  if (r < r1) add_bf16x8(acc, qh[static_cast<size_t>(r) * 8 + sub]);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
+    acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
+  }
+  __shared__ double wsum[8][kD];
+  if (lane < 8) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wsum[warp][8 * sub + i] = acc[i];
+  }
   __syncthreads();
   if (threadIdx.x < kD) {
     double t = 0.0;
-    for (int w = 0; w < 8; ++w) t += acc[w][threadIdx.x];
+    for (int w = 0; w < 8; ++w) t += wsum[w][threadIdx.x];
     partial[(static_cast<size_t>(hp) * gridDim.x + blockIdx.x) * kD + threadIdx.x] = t;
   }
 }
 
-// qbar = (sum of partials, in block order) / N, rounded once to fp32.
-__global__ void probe_mean_kernel(const double* __restrict__ partial, int nparts, int N,
-                                  float* __restrict__ qbar) {
-  const int hp = blockIdx.x, c = threadIdx.x;
-  double t = 0.0;
-  for (int b = 0; b < nparts; ++b) t += partial[(static_cast<size_t>(hp) * nparts + b) * kD + c];
-  qbar[hp * kD + c] = static_cast<float>(t / static_cast<double>(N));
+// qbar = (sum of partials) / N, rounded once to fp32.  Four threads per column take every
+// fourth partial; their sums are added in a fixed order.
+__global__ void __launch_bounds__(256) probe_mean_kernel(const double* __restrict__ partial, int nparts, int N,
+                                                         float* __restrict__ qbar) {
+  const int hp = blockIdx.x, c = threadIdx.x & (kD - 1), g = threadIdx.x >> 6;
+  const double* base = partial + static_cast<size_t>(hp) * nparts * kD + c;
+  double t0 = 0.0, t1 = 0.0;
+  int b = g;
+  for (; b + 4 < nparts; b += 8) {
+    t0 += base[static_cast<size_t>(b) * kD];
+    t1 += base[static_cast<size_t>(b + 4) * kD];
+  }
+  if (b < nparts) t0 += base[static_cast<size_t>(b) * kD];
+  __shared__ double gs[4][kD];
+  gs[g][c] = t0 + t1;
+  __syncthreads();
+  if (g == 0) qbar[hp * kD + c] = static_cast<float>(((gs[0][c] + gs[1][c]) + (gs[2][c] + gs[3][c])) /
+                                                    static_cast<double>(N));
 }
 
 // score_j = qbar . k_j / 8 (fp64 dot, fp32 result); special keys get -inf so they are never ranked.
+// Eight lanes per key row, each with one 16-byte chunk (a warp reads 4 whole rows, 512 contiguous
+// bytes, per load), two rows per lane group in flight; the 8 partial dots meet in 3 shuffles.
 __global__ void __launch_bounds__(256) probe_score_kernel(const uint16_t* __restrict__ k, int N, int V, int ns,
                                                           ProbeArgs a, const float* __restrict__ qbar,
                                                           float* __restrict__ scores) {
   const int hp = blockIdx.y;
   const int h = a.heads[hp];
-  const int lane = threadIdx.x & 31;
-  const double q0 = static_cast<double>(qbar[hp * kD + 2 * lane]);
-  const double q1 = static_cast<double>(qbar[hp * kD + 2 * lane + 1]);
-  const uint32_t* kh = reinterpret_cast<const uint32_t*>(k + static_cast<size_t>(h) * N * kD);
-  const int warps_total = gridDim.x * 8;
-  for (int j = blockIdx.x * 8 + (threadIdx.x >> 5); j < N; j += warps_total) {
-    const uint32_t w = kh[static_cast<size_t>(j) * (kD / 2) + lane];
-    double d = q0 * static_cast<double>(bf16_lo(w)) + q1 * static_cast<double>(bf16_hi(w));
+  const int sub = threadIdx.x & 7;
+  double qv[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-    if (lane == 0) {
-      const bool special = (j % V) < ns;
-      scores[static_cast<size_t>(hp) * N + j] = special ? -INFINITY : static_cast<float>(d * 0.125);
+  for (int i = 0; i < 8; ++i) qv[i] = static_cast<double>(qbar[hp * kD + 8 * sub + i]);
+  const uint4* kh = reinterpret_cast<const uint4*>(k + static_cast<size_t>(h) * N * kD);
+  const int groups = (gridDim.x * blockDim.x) >> 3;
+  for (int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 3; j < N; j += 2 * groups) {
+    const int j1 = j + groups;
+    const bool two = j1 < N;  // uniform over the 8 lanes of a row group
+    const uint4 w0 = kh[static_cast<size_t>(j) * 8 + sub];
+    const uint4 w1 = two ? kh[static_cast<size_t>(j1) * 8 + sub] : make_uint4(0u, 0u, 0u, 0u);
+    double x[8], d0 = 0.0, d1 = 0.0;
+    bf16x8_to_f64(w0, x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d0 = fma(qv[i], x[i], d0);
+    bf16x8_to_f64(w1, x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d1 = fma(qv[i], x[i], d1);
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      d0 += __shfl_xor_sync(0xffffffffu, d0, o);
+      d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+    }
+    if (sub == 0) {
+      scores[static_cast<size_t>(hp) * N + j] = (j % V) < ns ? -INFINITY : static_cast<float>(d0 * 0.125);
+      if (two) scores[static_cast<size_t>(hp) * N + j1] = (j1 % V) < ns ? -INFINITY : static_cast<float>(d1 * 0.125);
     }
   }
 }
@@ -200,16 +265,36 @@ __global__ void __launch_bounds__(128) dino_pool_kernel(const float* __restrict_
   __syncthreads();
   int count = 0;
   const int tok0 = t * kTile, tok1 = min(N, tok0 + kTile);
+  const int nc = dim >> 2;  // 16-byte chunks per feature row (dim is a multiple of 4, at most 1024)
   for (int tok = tok0 + warp; tok < tok1; tok += 4) {
     const int s = tok / V, loc = tok - s * V;
     if (loc < ns) continue;
-    const float* f = dino + (static_cast<size_t>(s) * P + (loc - ns)) * dim;
+    // the row once, in 16-byte loads, kept in registers for both passes
+    const float4* f = reinterpret_cast<const float4*>(dino + (static_cast<size_t>(s) * P + (loc - ns)) * dim);
+    float4 x[8];
     float ss = 0.f;
-    for (int c = lane; c < dim; c += 32) ss = fmaf(f[c], f[c], ss);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int i = 32 * c + lane;
+      x[c] = i < nc ? f[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      ss = fmaf(x[c].x, x[c].x, fmaf(x[c].y, x[c].y, fmaf(x[c].z, x[c].z, fmaf(x[c].w, x[c].w, ss))));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = 1.f / sqrtf(ss);
-    for (int c = lane; c < dim; c += 32) wsum[warp * dim + c] += f[c] * inv;
+    float4* w4 = reinterpret_cast<float4*>(wsum + warp * dim);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int i = 32 * c + lane;
+      if (i < nc) {
+        float4 a = w4[i];
+        a.x += x[c].x * inv;
+        a.y += x[c].y * inv;
+        a.z += x[c].z * inv;
+        a.w += x[c].w * inv;
+        w4[i] = a;
+      }
+    }
   }
   for (int tok = tok0; tok < tok1; ++tok) count += ((tok % V) >= ns);
   __syncthreads();
@@ -1053,8 +1138,10 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
       a.cache_off[i] = sp.probe_off[i];
     }
     probe_partial_kernel<<<dim3(kProbePartials, sp.n_probe), 256, 0, stream>>>(q, sp.N, a, partial);
-    probe_mean_kernel<<<sp.n_probe, kD, 0, stream>>>(partial, kProbePartials, sp.N, qbar);
-    probe_score_kernel<<<dim3(296, sp.n_probe), 256, 0, stream>>>(k, sp.N, sp.V, sp.ns, a, qbar, scores);
+    probe_mean_kernel<<<sp.n_probe, 4 * kD, 0, stream>>>(partial, kProbePartials, sp.N, qbar);
+    // 32 key rows per 256-thread block and step; at most 8 blocks per SM and head
+    const int score_blocks = std::max(1, std::min((sp.N + 63) / 64, 8 * sp.num_sms));
+    probe_score_kernel<<<dim3(score_blocks, sp.n_probe), 256, 0, stream>>>(k, sp.N, sp.V, sp.ns, a, qbar, scores);
     probe_topk_kernel<<<sp.n_probe, 1024, 0, stream>>>(scores, sp.N, a, cache);
     *n_launch += 4;
   }

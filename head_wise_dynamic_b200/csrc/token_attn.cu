@@ -1,16 +1,19 @@
-// Attention of token-wise correspondence heads: every query row keeps its own keys.
+// Attention of the patch queries of token-wise correspondence heads: every such query row keeps
+// its own keys.
 //
 // SAF3R ("SAF3R: Dynamic Sparse Attention for Feed-Forward 3D Reconstruction Transformers"),
 // section 4.1, "DINO Top-K Kernel": a patch query keeps, in every frame, the Top-K patch tokens
 // most similar to it in DINO features (section 5.1: K per frame), here plus every special
-// token; a special-token query has no DINO feature and keeps every key.  Exact softmax over the
-// kept keys (logit -inf elsewhere), scale 1/sqrt(64).
+// token.  Exact softmax over the kept keys (logit -inf elsewhere), scale 1/sqrt(64).  (A
+// special-token query has no DINO feature and keeps every key: those rows are dense and run in
+// the tensor-core attention kernel.)
 //
-// No two query rows share a key set, so there is no dense block for the tensor cores: one warp
-// per query row, split into 8 groups of 4 lanes; a group takes every 8th kept key, each lane
-// of it 16 of the 64 features (a 128-byte K row and V row gathered from L2 by one group in one
-// coalesced access each).  A group keeps its own running max, sum and accumulator in fp32; the
-// 8 group states are merged at the end and the warp stores the row with one coalesced access.
+// No two patch query rows share a key set, so there is no dense block for the tensor cores: one
+// warp per query row, split into 8 groups of 4 lanes; a group takes kept keys n, n + 8 together
+// (every 16th pair), each lane of it 16 of the 64 features (a 128-byte K row and V row gathered
+// from L2 by one group in one coalesced access each; both keys' K and V rows are requested
+// before any of them is used).  A group keeps its own running max, sum and accumulator in fp32;
+// the 8 group states are merged at the end and the warp stores the row with one coalesced access.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -45,6 +48,20 @@ __device__ __forceinline__ int special_tok(int r, int V, int ns) {
   return s * V + (r - s * ns);
 }
 
+// Token of kept key n of a patch query: ranks n < nl come from the per-frame lists (frame n / kf),
+// the rest are the special tokens.  An out-of-range list entry is recorded in the error word and
+// read as patch 0 (the group stays converged).
+__device__ __forceinline__ int key_token(const TokenAttnParams& p, const int32_t* lists, int n, int nl, int kf) {
+  if (n >= nl) return special_tok(n - nl, p.V, p.ns);
+  const int s = n / kf, r = n - s * kf;
+  int pp = lists[s * p.tok_kmax + r];
+  if (pp < 0 || pp >= p.P) {
+    atomicCAS(p.err, 0, SAF3R_ERR_INDEX);
+    pp = 0;
+  }
+  return s * p.V + p.ns + pp;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(256) token_attn_kernel(const TokenAttnParams p) {
@@ -53,65 +70,61 @@ __global__ void __launch_bounds__(256) token_attn_kernel(const TokenAttnParams p
   const int grp = lane >> 2, sub = lane & 3;            // key group, feature quarter [16*sub, 16*sub+16)
   const unsigned gmask = 0xFu << (grp * 4);
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long total = static_cast<long long>(p.n_heads) * p.N;
+  const int R = p.S * p.P;  // patch query rows of a head (its special rows run in the tensor-core kernel)
+  const long long total = static_cast<long long>(p.n_heads) * R;
   const int nsp = p.ns * p.S;
   for (long long task = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; task < total;
        task += warps) {
-    const int hi = static_cast<int>(task / p.N);
-    const int i = static_cast<int>(task - static_cast<long long>(hi) * p.N);
+    const int hi = static_cast<int>(task / R);
+    const int a = static_cast<int>(task - static_cast<long long>(hi) * R);  // patch row a = s*P + patch
+    const int i = (a / p.P) * p.V + p.ns + (a % p.P);
     const int h = p.heads[hi], kf = p.k[hi];  // kf: per-frame budget of this head
     const size_t hb = static_cast<size_t>(h) * p.N * kD;
-    const int s_i = i / p.V, loc = i - s_i * p.V;
-    const bool special = loc < p.ns;
-    const int nk = special ? p.N : p.S * kf + nsp;
-    const int32_t* lists =
-        special ? nullptr
-                : p.cache + p.tok_off + (static_cast<size_t>(s_i) * p.P + (loc - p.ns)) * p.S * p.tok_kmax;
+    const int nl = p.S * kf;  // ranked keys; the special tokens follow
+    const int nk = nl + nsp;
+    const int32_t* lists = p.cache + p.tok_off + static_cast<size_t>(a) * p.S * p.tok_kmax;
     float qv[16];
     load16(p.q + hb + static_cast<size_t>(i) * kD + 16 * sub, qv);
     float m = -INFINITY, l = 0.f;
     float o[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) o[c] = 0.f;
-    for (int n = grp; n < nk; n += 8) {
-      int tok;
-      if (special) {
-        tok = n;
-      } else if (n < p.S * kf) {
-        const int s = n / kf, r = n - s * kf;
-        int pp = lists[s * p.tok_kmax + r];
-        if (pp < 0 || pp >= p.P) {
-          atomicCAS(p.err, 0, SAF3R_ERR_INDEX);
-          pp = 0;  // keep the group converged; the error word reports the bad index
-        }
-        tok = s * p.V + p.ns + pp;
-      } else {
-        tok = special_tok(n - p.S * kf, p.V, p.ns);
-      }
-      float kv[16];
-      load16(p.k_ + hb + static_cast<size_t>(tok) * kD + 16 * sub, kv);
-      float d0 = 0.f, d1 = 0.f;
+    for (int n = grp; n < nk; n += 16) {
+      const bool two = n + 8 < nk;
+      const int tok0 = key_token(p, lists, n, nl, kf);
+      const int tok1 = two ? key_token(p, lists, n + 8, nl, kf) : tok0;
+      float k0[16], k1[16], v0[16], v1[16];
+      load16(p.k_ + hb + static_cast<size_t>(tok0) * kD + 16 * sub, k0);
+      load16(p.k_ + hb + static_cast<size_t>(tok1) * kD + 16 * sub, k1);
+      load16(p.v + hb + static_cast<size_t>(tok0) * kD + 16 * sub, v0);
+      load16(p.v + hb + static_cast<size_t>(tok1) * kD + 16 * sub, v1);
+      float d0 = 0.f, d1 = 0.f, e0 = 0.f, e1 = 0.f;
 #pragma unroll
       for (int c = 0; c < 16; c += 2) {
-        d0 = fmaf(qv[c], kv[c], d0);
-        d1 = fmaf(qv[c + 1], kv[c + 1], d1);
+        d0 = fmaf(qv[c], k0[c], d0);
+        d1 = fmaf(qv[c + 1], k0[c + 1], d1);
+        e0 = fmaf(qv[c], k1[c], e0);
+        e1 = fmaf(qv[c + 1], k1[c + 1], e1);
       }
-      float d = d0 + d1;
-      d += __shfl_xor_sync(gmask, d, 1);
-      d += __shfl_xor_sync(gmask, d, 2);
-      const float x = d * kLog2eOver8;
-      if (x > m + kThresh || m == -INFINITY) {
-        const float alpha = m == -INFINITY ? 0.f : fast_exp2(m - x);
+      float x0 = d0 + d1, x1 = e0 + e1;
+      x0 += __shfl_xor_sync(gmask, x0, 1);
+      x1 += __shfl_xor_sync(gmask, x1, 1);
+      x0 += __shfl_xor_sync(gmask, x0, 2);
+      x1 += __shfl_xor_sync(gmask, x1, 2);
+      x0 *= kLog2eOver8;
+      x1 = two ? x1 * kLog2eOver8 : -INFINITY;
+      const float xm = fmaxf(x0, x1);
+      if (xm > m + kThresh || m == -INFINITY) {
+        const float alpha = m == -INFINITY ? 0.f : fast_exp2(m - xm);
         l *= alpha;
 #pragma unroll
         for (int c = 0; c < 16; ++c) o[c] *= alpha;
-        m = x;
+        m = xm;
       }
-      const float pw = fast_exp2(x - m);
-      l += pw;
-      load16(p.v + hb + static_cast<size_t>(tok) * kD + 16 * sub, kv);
+      const float w0 = fast_exp2(x0 - m), w1 = fast_exp2(x1 - m);
+      l += w0 + w1;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) o[c] = fmaf(pw, kv[c], o[c]);
+      for (int c = 0; c < 16; ++c) o[c] = fmaf(w1, v1[c], fmaf(w0, v0[c], o[c]));
     }
     // merge the 8 group states (lanes of one feature quarter: xor over lane bits 2..4)
     float mm = m;

@@ -429,12 +429,11 @@ def nmse_table_sampled(L, candidates, Q, K, V, dino, rows_per_head) -> np.ndarra
     sample it is the sample estimate (parity unpinned at full size)."""
     H = Q.shape[0]
     table = np.zeros((H, len(candidates)), dtype=np.float64)
+    full = [dense_rows(Q[h], K[h], V[h], rows_per_head[h]) for h in range(H)]  # O_full, once per head
     for c, cand in enumerate(candidates):
         heads = [apply_candidate(cand, h) for h in range(H)]
         sel = select(L, heads, Q, K, dino)
         for h in range(H):
-            rows = rows_per_head[h]
-            of = dense_rows(Q[h], K[h], V[h], rows)
-            os_ = sparse_rows(L, heads[h], sel, h, Q[h], K[h], V[h], rows)
-            table[h, c] = nmse(of, os_)
+            os_ = sparse_rows(L, heads[h], sel, h, Q[h], K[h], V[h], rows_per_head[h])
+            table[h, c] = nmse(full[h], os_)
     return table

@@ -132,6 +132,10 @@ WORKLOADS = {
     "s32_token": Workload("s32_token", Layout(S=32, g=37, H=16), M=4096, delta=97, D=1024,
                           heads=[HeadCfg(TOKEN, k=16)] * 4 + _split16(4096, 32, 10)[4:],
                           sample_rows=256, seed=SEED_BASE + 1000),
+    # the S=100 layer with its position heads replaced by token-wise per-frame DINO Top-16 heads
+    "s100_token": Workload("s100_token", Layout(S=100, g=37, H=16), M=4096, delta=97, D=1024,
+                           heads=[HeadCfg(TOKEN, k=16)] * 4 + _split16(8192, 64, 16)[4:],
+                           calls=4, sample_rows=128, seed=SEED_BASE + 2000),
     # the S=100 layer with its correspondence heads as tile Top-64 united with a stride-32 lattice
     "s100_hybrid": Workload("s100_hybrid", Layout(S=100, g=37, H=16), M=4096, delta=97, D=1024,
                             heads=_split16(8192, 64, 16)[:8] +

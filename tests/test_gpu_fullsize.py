@@ -6,7 +6,7 @@ import pytest
 
 import oracle as O
 from saf3r_synth import WORKLOADS, Scene, bf16_to_f32, qkv, sample_rows
-from parity_util import HeadSelections, check_probe, check_tiles, compare_outputs
+from parity_util import HeadSelections, check_probe, check_tiles, check_token_lists, compare_outputs
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -29,6 +29,11 @@ def _check_layer(wl, att, scene, layer, rows_per_head, sels=None):
             elif hc.kind in (O.CORR, O.HYBRID):  # ranked tiles
                 ranked = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(L.T, hc.k)
                 sels.accept(L, h, hc, ranked, check_tiles(ranked, sels.base, hc.k, f"tile head {h}"))
+            elif hc.kind == O.TOKEN:  # per-frame lists of the rows that are checked below
+                lists = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).reshape(L.S * L.P, L.S, hc.k)
+                rows = sample_rows(wl, h, rows_per_head, seed_extra=layer)
+                sels.accept(L, h, hc, lists, check_token_lists(lists, L, sels.base.unit, hc.k, rows,
+                                                               f"token head {h}"))
     att.out.fill_(float("nan"))
     out = att(q, k, v)
     torch.cuda.synchronize()
@@ -68,3 +73,14 @@ def test_s100_hybrid_layer():
     scene = Scene(wl)
     att = hw.SparseGlobalAttention(wl.layout, wl.heads)
     _check_layer(wl, att, scene, 0, 512)
+
+
+def test_s100_token_layer():
+    """The S=100 layer with per-frame Top-16 token-wise heads in place of the position heads:
+    sampled rows (the special-token rows among them run in the tensor-core kernel as dense rows,
+    the patch rows in the gather kernel) and their per-frame lists against the oracle."""
+    import head_wise_dynamic_b200 as hw
+    wl = WORKLOADS["s100_token"]
+    scene = Scene(wl)
+    att = hw.SparseGlobalAttention(wl.layout, wl.heads)
+    _check_layer(wl, att, scene, 0, 96)

@@ -318,3 +318,26 @@ def test_s32_token_heads_sampled_rows(s32):
     rows = {h: sample_rows(s32.wl, h, 64) for h in range(4)}
     _check_token_heads(s32, heads, att, sels, lambda h: rows[h])
     check_rows(s32, heads, sels, out, lambda h: rows[h] if h < 4 else sample_rows(s32.wl, h, 128))
+
+
+# ---------------------------------------------------------------- running-max growth
+
+def test_growing_logits_rescale_the_accumulator():
+    """Every query gets q_0 = 8 and key j gets k_0 = 7 * floor(3j / N), so the logits of the middle
+    and last third of the token sequence are raised by 7 and 14 (natural units, about 10 and 20
+    in log2 units, each past the kernel's stale-max threshold of 8): every row's running max jumps
+    twice, inside blocks as well as between them, and the accumulator and the partly written P
+    are rescaled.  The softmax stays spread over a third of the keys (bf16 P rounding averages
+    out).  All rows of every head kind against the oracle."""
+    heads = [HeadCfg(PROBE, k=300), HeadCfg(SCAN, stride=2, phase=1), HeadCfg(DENSE), HeadCfg(POSITION),
+             HeadCfg(CORR, k=6)]
+    case = Case(_custom(4, 16, heads, seed=91))
+    L = case.L
+    step = torch.div(torch.arange(L.N, device="cuda") * 3, L.N, rounding_mode="floor").to(torch.float32)
+    case.q[:, :, 0] = 8.0
+    case.k[:, :, 0] = (7.0 * step).to(torch.bfloat16).view(1, L.N)
+    case.Q, case.K = bf16_to_f32(case.q), bf16_to_f32(case.k)
+    att, out = run_gpu(case, heads)
+    sel = oracle_select(case, heads)
+    sels = check_selection(case, heads, att, sel)
+    check_rows(case, heads, sels, out, lambda h: np.arange(L.N))
