@@ -37,12 +37,11 @@ L2_NOTE = "inputs larger than L2 (Q/K/V 3 x 281 MB per call)"
 
 
 # DRAM traffic of one attention launch on this workload, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
-# source it was taken on: a changed kernel reports null until it is re-captured.
-# Taken on the S=32-view call (189,911,040 + 70,724,864 bytes) and scaled to the
-# S=100-view call by the token count (137,400 / 43,968): Q/K/V/O bytes grow with N.
-ATTN_TRAFFIC = {"kernel_source_sha256": "e2e396f8a6f69c8e77ff2033b0fd65a1af3eff36fd75a61f75592c953a9fcd45",
-                "bytes_per_launch": round((189911040 + 70724864) * 137400 / 43968), "workload": "s100"}
+# (dram__bytes_read.sum + dram__bytes_write.sum of one S=100-view layer call, one launch, a
+# 1-pass metric set; profiles/attn_sm100_s100_dram.md), valid only for the kernel source it was
+# taken on: a changed kernel reports null until it is re-captured.
+ATTN_TRAFFIC = {"kernel_source_sha256": "011c36a96a2e15970abebf1d18f437a2ba56f66200d43960a5bc0e9e35e1f6f3",
+                "bytes_per_launch": 598700544 + 264559872, "workload": "s100"}
 
 
 def kernel_source_sha256():
