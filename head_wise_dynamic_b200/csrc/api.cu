@@ -307,7 +307,7 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
         l.seg_begin = s.seg_total;
         l.cnt_begin = s.cnt_total;
         s.seg_total += static_cast<long long>(l.cap) * l.n_items;
-        s.cnt_total += l.n_items;
+        s.cnt_total += 2 * l.n_items;  // per item: segments, then 128-key blocks
         s.lists.push_back(l);
         found = static_cast<int>(s.lists.size()) - 1;
       }

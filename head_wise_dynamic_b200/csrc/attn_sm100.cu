@@ -55,6 +55,7 @@ constexpr int kThreads = 384;
 constexpr int kStages = 4;
 constexpr int kTileBytes = 128 * 64 * 2;  // 128 rows x 64 bf16
 constexpr int kHalfBytes = 64 * 64 * 2;   // 64 rows x 64 bf16
+constexpr int kSegBuf = 1024;             // key runs of one item staged in shared memory (longer lists are read in place)
 constexpr float kScaleLog2 = 0.18033688011112042f;  // log2(e) / sqrt(64)
 constexpr float kRescaleThreshold = 8.0f;           // log2 units: keep a stale max until it is 256x off
 // Pairs (of the 32 per 64-key half-block) whose exponentials run on the FMA pipe: bit i = pair i.
@@ -81,6 +82,7 @@ struct AttnSmem {
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_full[2], o_done[2];
   Half info[kStages][2];      // the key halves of the block in each K/V stage (written by the producer)
+  Seg segbuf[kSegBuf];        // the current item's key runs (copied by the producer warp, read by its lane 0)
   uint64_t pair[4];           // the two warps sharing rows 32*w..+31 (w = warp % 4) meet here at an item's end
   float stats[2][2][128][2];  // [key half][tile][row] = (running max, running sum) for the final merge
   uint32_t tmem_base;
@@ -139,13 +141,14 @@ __device__ __forceinline__ ItemInfo item_info(const AttnParams& p, int item) {
   if (hp.seg_list < 0) {
     it.w.list = nullptr;
     it.w.nseg = 1;
+    it.nblk = (((hp.seg.len + 63) >> 6) + 1) >> 1;
   } else {
+    // the plan stored the item's segment and block counts side by side
     it.w.list = p.segs + hp.seg_list + static_cast<long long>(it.local) * hp.seg_cap;
-    it.w.nseg = p.seg_counts[hp.cnt_list + it.local];
+    const int2 c = *reinterpret_cast<const int2*>(p.seg_counts + hp.cnt_list + 2 * it.local);
+    it.w.nseg = c.x;
+    it.nblk = c.y;
   }
-  int nhb = 0;
-  for (int i = 0; i < it.w.nseg; ++i) nhb += (it.w.seg_at(i).len + 63) >> 6;
-  it.nblk = (nhb + 1) >> 1;
   return it;
 }
 
@@ -182,63 +185,86 @@ __device__ __forceinline__ int mapped_tile(const AttnParams& p, const HeadPlan& 
   return i < p.T ? p.qmap[hp.q_base + i] : -1;
 }
 
-// ------------------------------------------------------------------ TMA producer (one thread)
+// One item's loads (lane 0 of the producer warp): the Q tiles, then every 128-key block's K and V
+// halves into the ring.  Returns false when a wait gave up.
+__device__ __forceinline__ bool producer_item(const AttnParams& p, AttnSmem& sm, const CUtensorMap& tmQ,
+                                              const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                              const CUtensorMap& tmQC, const CUtensorMap& tmKC,
+                                              const CUtensorMap& tmVC, ItemInfo& it, const HeadPlan& hp,
+                                              uint32_t& k_issued, uint32_t& v_issued, uint32_t& q_issued) {
+  volatile int* abort = &sm.abort;
+  const long long budget = p.wait_budget;
+  if (q_issued > 0 && !mbar_wait(&sm.q_empty, (q_issued - 1) & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))
+    return false;
+  mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
+  for (int quarter = 0; quarter < 4; ++quarter) {
+    void* dst = sm.q[quarter >> 1] + (quarter & 1) * kHalfBytes;
+    if (hp.q_src == 1 || hp.q_src == 3) {
+      tma_load_2d(dst, &tmQC, 0, hp.q_base + it.q0 + quarter * 64, &sm.q_full);
+    } else {
+      int row = it.q0 + quarter * 64;
+      if (hp.q_src == 2) {
+        const int u = mapped_tile(p, hp, it.local, quarter);
+        row = u >= 0 ? u * 64 : -64;  // past the last tile: an all-zero box
+      }
+      tma_load_3d(dst, &tmQ, 0, row, hp.head, &sm.q_full);
+    }
+  }
+  ++q_issued;
+  for (int b = 0; b < it.nblk; ++b) {
+    const Half h0 = it.w.next();
+    const Half h1 = it.w.next();
+    const uint32_t stage = k_issued % kStages, ph = (k_issued / kStages) & 1;
+    if (k_issued >= kStages && !mbar_wait(&sm.k_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))
+      return false;
+    mbar_arrive_expect_tx(&sm.k_full[stage], kTileBytes);
+    if (h0.have) load_half(hp, h0, sm.k[stage], &tmK, &tmKC, &sm.k_full[stage]); else tma_load_3d(sm.k[stage], &tmK, 0, -64, hp.head, &sm.k_full[stage]);
+    if (h1.have) load_half(hp, h1, sm.k[stage] + kHalfBytes, &tmK, &tmKC, &sm.k_full[stage]); else tma_load_3d(sm.k[stage] + kHalfBytes, &tmK, 0, -64, hp.head, &sm.k_full[stage]);
+    ++k_issued;
+    if (v_issued >= kStages && !mbar_wait(&sm.v_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))
+      return false;
+    // the block's halves for the softmax warps; the arrival below releases them with the stage
+    sm.info[stage][0] = h0;
+    sm.info[stage][1] = h1;
+    mbar_arrive_expect_tx(&sm.v_full[stage], kTileBytes);
+    if (h0.have) load_half(hp, h0, sm.v[stage], &tmV, &tmVC, &sm.v_full[stage]); else tma_load_3d(sm.v[stage], &tmV, 0, -64, hp.head, &sm.v_full[stage]);
+    if (h1.have) load_half(hp, h1, sm.v[stage] + kHalfBytes, &tmV, &tmVC, &sm.v_full[stage]); else tma_load_3d(sm.v[stage] + kHalfBytes, &tmV, 0, -64, hp.head, &sm.v_full[stage]);
+    ++v_issued;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ TMA producer (one warp, lane 0 issues)
+//
+// At each item the whole warp copies the item's key runs into shared memory (a list head's runs
+// would otherwise be read one by one from global memory as lane 0 walks them); lane 0 then walks
+// them and issues every load.
 __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm, const CUtensorMap& tmQ,
                                               const CUtensorMap& tmK, const CUtensorMap& tmV,
                                               const CUtensorMap& tmQC, const CUtensorMap& tmKC,
-                                              const CUtensorMap& tmVC) {
+                                              const CUtensorMap& tmVC, int lane) {
   volatile int* abort = &sm.abort;
   const long long budget = p.wait_budget;
-  tma_prefetch_desc(&tmQ);
-  tma_prefetch_desc(&tmK);
-  tma_prefetch_desc(&tmV);
+  if (lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
   uint32_t k_issued = 0, v_issued = 0, q_issued = 0;
   bool ok = true;
   for (int item = blockIdx.x; ok && item < p.total_items; item += gridDim.x) {
     ItemInfo it = item_info(p, item);
     const HeadPlan& hp = p.heads[it.hi];
-    if (q_issued > 0 && !mbar_wait(&sm.q_empty, (q_issued - 1) & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) break;
-    mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
-    for (int quarter = 0; quarter < 4; ++quarter) {
-      void* dst = sm.q[quarter >> 1] + (quarter & 1) * kHalfBytes;
-      if (hp.q_src == 1 || hp.q_src == 3) {
-        tma_load_2d(dst, &tmQC, 0, hp.q_base + it.q0 + quarter * 64, &sm.q_full);
-      } else {
-        int row = it.q0 + quarter * 64;
-        if (hp.q_src == 2) {
-          const int u = mapped_tile(p, hp, it.local, quarter);
-          row = u >= 0 ? u * 64 : -64;  // past the last tile: an all-zero box
-        }
-        tma_load_3d(dst, &tmQ, 0, row, hp.head, &sm.q_full);
-      }
+    if (it.w.list != nullptr && it.w.nseg <= kSegBuf) {
+      for (int i = lane; i < it.w.nseg; i += 32) sm.segbuf[i] = it.w.list[i];
+      it.w.list = sm.segbuf;
     }
-    ++q_issued;
-    for (int b = 0; b < it.nblk; ++b) {
-      const Half h0 = it.w.next();
-      const Half h1 = it.w.next();
-      const uint32_t stage = k_issued % kStages, ph = (k_issued / kStages) & 1;
-      if (k_issued >= kStages && !mbar_wait(&sm.k_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) {
-        ok = false;
-        break;
-      }
-      mbar_arrive_expect_tx(&sm.k_full[stage], kTileBytes);
-      if (h0.have) load_half(hp, h0, sm.k[stage], &tmK, &tmKC, &sm.k_full[stage]); else tma_load_3d(sm.k[stage], &tmK, 0, -64, hp.head, &sm.k_full[stage]);
-      if (h1.have) load_half(hp, h1, sm.k[stage] + kHalfBytes, &tmK, &tmKC, &sm.k_full[stage]); else tma_load_3d(sm.k[stage] + kHalfBytes, &tmK, 0, -64, hp.head, &sm.k_full[stage]);
-      ++k_issued;
-      if (v_issued >= kStages && !mbar_wait(&sm.v_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)) {
-        ok = false;
-        break;
-      }
-      // the block's halves for the softmax warps; the arrival below releases them with the stage
-      sm.info[stage][0] = h0;
-      sm.info[stage][1] = h1;
-      mbar_arrive_expect_tx(&sm.v_full[stage], kTileBytes);
-      if (h0.have) load_half(hp, h0, sm.v[stage], &tmV, &tmVC, &sm.v_full[stage]); else tma_load_3d(sm.v[stage], &tmV, 0, -64, hp.head, &sm.v_full[stage]);
-      if (h1.have) load_half(hp, h1, sm.v[stage] + kHalfBytes, &tmV, &tmVC, &sm.v_full[stage]); else tma_load_3d(sm.v[stage] + kHalfBytes, &tmV, 0, -64, hp.head, &sm.v_full[stage]);
-      ++v_issued;
-    }
+    __syncwarp();
+    if (lane == 0) ok = producer_item(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, it, hp, k_issued, v_issued, q_issued);
+    ok = __shfl_sync(0xffffffffu, ok, 0);  // the runs are not overwritten before lane 0 has walked them
   }
-  // Teardown: every copy this thread issued must have landed before the CTA exits
+  if (lane != 0) return;
+  // Teardown: every copy lane 0 issued must have landed before the CTA exits
   // (these waits ignore the abort flag but stay bounded).
   const long long drain = kDrainBudget;
   if (q_issued > 0) mbar_wait_drain(&sm.q_full, (q_issued - 1) & 1, drain);
@@ -817,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) reg_dealloc_dec<104>();  // 104*128 + 200*256 = 168*384 registers
   if (warp == 0) {
-    if (lane == 0) producer_role(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC);
+    producer_role(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, lane);
     __syncwarp();
   } else if (warp == 1) {
     mma_role(p, sm, tmem);

@@ -82,7 +82,7 @@ struct HeadPlan {
   int32_t item_begin; // first global item index
   int32_t seg_list;   // -1: one implicit segment (below); else Seg offset of item 0's list
   int32_t seg_cap;    // Seg entries per item
-  int32_t cnt_list;   // offset of the per-item segment counts
+  int32_t cnt_list;   // offset of the per-item counts: [2*item] segments, [2*item + 1] 128-key blocks
   Seg seg;            // implicit segment
   int32_t radius;     // position heads
   int32_t nb_base;    // position heads: derived row where the cell-major neighbour rows start

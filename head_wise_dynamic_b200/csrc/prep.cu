@@ -190,7 +190,10 @@ __global__ void plan_position_kernel(int n_items, int S, int gh, int gw, int ns,
       }
     }
   }
-  counts[m] = n;
+  int nhb = 0;  // 64-key half-blocks of the item's runs
+  for (int x = 0; x < n; ++x) nhb += (out[x].len + 63) >> 6;
+  counts[2 * m] = n;
+  counts[2 * m + 1] = (nhb + 1) >> 1;
 }
 
 // Key runs of every 256-row item of a correspondence head: the union of its four
@@ -259,7 +262,8 @@ __global__ void __launch_bounds__(256) plan_corr_kernel(const int32_t* __restric
   if (threadIdx.x == 0) {
     const int nu = min(base, cap - 1);
     out[nu] = Seg{1, 0, tail_len, kSegAllQuarters};  // the head's derived rows: specials (and its lattice)
-    counts[m] = nu + 1;
+    counts[2 * m] = nu + 1;
+    counts[2 * m + 1] = (nu + ((tail_len + 63) >> 6) + 1) >> 1;  // each key tile is one half-block
   }
 }
 
