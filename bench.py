@@ -40,8 +40,8 @@ L2_NOTE = "inputs larger than L2 (Q/K/V 3 x 281 MB per call)"
 # (dram__bytes_read.sum + dram__bytes_write.sum of one S=100-view layer call, one launch, a
 # 1-pass metric set; profiles/attn_sm100_s100_dram.md), valid only for the kernel source it was
 # taken on: a changed kernel reports null until it is re-captured.
-ATTN_TRAFFIC = {"kernel_source_sha256": "011c36a96a2e15970abebf1d18f437a2ba56f66200d43960a5bc0e9e35e1f6f3",
-                "bytes_per_launch": 598700544 + 264559872, "workload": "s100"}
+ATTN_TRAFFIC = {"kernel_source_sha256": "8a3e7a5a9a5b8aec2e0b0f2611aebf447492138bd3fcf39fb73328ce603aa400",
+                "bytes_per_launch": 618848256 + 265734912, "workload": "s100"}
 
 
 def kernel_source_sha256():
