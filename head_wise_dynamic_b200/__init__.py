@@ -183,7 +183,7 @@ def saf3r_select_kv(layout, cfg, q, k, dino, cache, workspace, stream=None):
 
 def saf3r_select_kv_static(layout, cfg, q, k, dino, cache, stream=None):
     """saf3r_select_kv for callers that cannot allocate a device workspace: the scratch
-    comes from a fixed 16 MiB array inside the library (see include/saf3r.h for the limit,
+    comes from a fixed 40 MiB array inside the library (see include/saf3r.h for the limit,
     the first-call set-up and the rule that overlapping calls race)."""
     f = lib().saf3r_select_kv_static
     f.argtypes = [ctypes.POINTER(saf3r_layout), ctypes.POINTER(saf3r_head_cfg)] + [ctypes.c_void_p] * 5

@@ -21,15 +21,16 @@ namespace saf3r {
 namespace {
 
 constexpr int kProbePartials = 296;  // row blocks per probe head (2 x 148 SMs)
+#ifndef SAF3R_PROBE_ROWS_IN_FLIGHT
+#define SAF3R_PROBE_ROWS_IN_FLIGHT 4
+#endif
+constexpr int kProbeRowsInFlight = SAF3R_PROBE_ROWS_IN_FLIGHT;  // 16-byte loads per lane before use
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   // monotone map fp32 -> uint32 (larger float -> larger key)
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 struct ProbeArgs {
   int n_probe;
@@ -38,34 +39,45 @@ struct ProbeArgs {
   int cache_off[kMaxHeads];  // int32 offset of the key list in the cache
 };
 
-// The 8 bf16 features of a 16-byte chunk as fp64, in order.
-__device__ __forceinline__ void bf16x8_to_f64(const uint4& w, double (&x)[8]) {
-  x[0] = static_cast<double>(bf16_lo(w.x));
-  x[1] = static_cast<double>(bf16_hi(w.x));
-  x[2] = static_cast<double>(bf16_lo(w.y));
-  x[3] = static_cast<double>(bf16_hi(w.y));
-  x[4] = static_cast<double>(bf16_lo(w.z));
-  x[5] = static_cast<double>(bf16_hi(w.z));
-  x[6] = static_cast<double>(bf16_lo(w.w));
-  x[7] = static_cast<double>(bf16_hi(w.w));
+// bf16 -> fp64 without a conversion instruction.  A bf16 is the top half of an fp32 (sign, 8-bit
+// exponent, 7-bit mantissa).  Placed in the high word of a double with the exponent zero-extended
+// to 11 bits, its bits read as x * 2^-896 exactly: for a normal x the exponent bias becomes 1023
+// instead of 127, and a subnormal x stays subnormal with the same scale (finite x only).  Sums and
+// products of such scaled values round exactly as those of the unscaled ones in the same order
+// (a power-of-two scale commutes with rounding while the result is normal; below that, every sum
+// of bf16 values is a multiple of 2^-133 and exact either way).
+constexpr double kBf16Unscale = 0x1p896;
+__device__ __forceinline__ double bf16_lo_scaled(uint32_t w) {
+  return __hiloint2double(static_cast<int>(((w & 0x8000u) << 16) | ((w & 0x7FFFu) << 13)), 0);
+}
+__device__ __forceinline__ double bf16_hi_scaled(uint32_t w) {
+  return __hiloint2double(static_cast<int>((w & 0x80000000u) | ((w & 0x7FFF0000u) >> 3)), 0);
 }
 
-// acc[i] += feature i of a 16-byte chunk of 8 bf16 features (fp64 sums).
+// The 8 bf16 features of a 16-byte chunk as fp64 scaled by 2^-896, in order.
+__device__ __forceinline__ void bf16x8_to_f64(const uint4& w, double (&x)[8]) {
+  x[0] = bf16_lo_scaled(w.x);
+  x[1] = bf16_hi_scaled(w.x);
+  x[2] = bf16_lo_scaled(w.y);
+  x[3] = bf16_hi_scaled(w.y);
+  x[4] = bf16_lo_scaled(w.z);
+  x[5] = bf16_hi_scaled(w.z);
+  x[6] = bf16_lo_scaled(w.w);
+  x[7] = bf16_hi_scaled(w.w);
+}
+
+// acc[i] += feature i of a 16-byte chunk of 8 bf16 features (fp64 sums, scaled by 2^-896).
 __device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4& w) {
-  acc[0] += static_cast<double>(bf16_lo(w.x));
-  acc[1] += static_cast<double>(bf16_hi(w.x));
-  acc[2] += static_cast<double>(bf16_lo(w.y));
-  acc[3] += static_cast<double>(bf16_hi(w.y));
-  acc[4] += static_cast<double>(bf16_lo(w.z));
-  acc[5] += static_cast<double>(bf16_hi(w.z));
-  acc[6] += static_cast<double>(bf16_lo(w.w));
-  acc[7] += static_cast<double>(bf16_hi(w.w));
+  double x[8];
+  bf16x8_to_f64(w, x);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] += x[i];
 }
 
 // Partial fp64 column sums of Q_h over a range of rows.  Lane l of a warp reads the 16-byte
 // chunk (l % 8) of row r + l / 8 (a warp reads 4 whole rows, 512 contiguous bytes, per load) and
-// keeps the 8 column sums of its chunk; two rows per lane are in flight per step.  The lanes and
-// warps that share a chunk are added in a fixed order at the end.
+// keeps the 8 column sums of its chunk; kProbeRowsInFlight rows per lane are loaded before any is
+// added.  The lanes and warps that share a chunk are added in a fixed order at the end.
 __global__ void __launch_bounds__(256) probe_partial_kernel(const uint16_t* __restrict__ q, int N,
                                                             ProbeArgs a, double* __restrict__ partial) {
   const int hp = blockIdx.y;
@@ -79,13 +91,14 @@ __global__ void __launch_bounds__(256) probe_partial_kernel(const uint16_t* __re
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0;
   int r = r0 + warp * 4 + (lane >> 3);
-  for (; r + 32 < r1; r += 64) {
-    const uint4 w0 = qh[static_cast<size_t>(r) * 8 + sub];
-    const uint4 w1 = qh[static_cast<size_t>(r + 32) * 8 + sub];
-    add_bf16x8(acc, w0);
-    add_bf16x8(acc, w1);
+  for (; r + 32 * (kProbeRowsInFlight - 1) < r1; r += 32 * kProbeRowsInFlight) {
+    uint4 w[kProbeRowsInFlight];
+#pragma unroll
+    for (int f = 0; f < kProbeRowsInFlight; ++f) w[f] = qh[static_cast<size_t>(r + 32 * f) * 8 + sub];
+#pragma unroll
+    for (int f = 0; f < kProbeRowsInFlight; ++f) add_bf16x8(acc, w[f]);
   }
-  if (r < r1) add_bf16x8(acc, qh[static_cast<size_t>(r) * 8 + sub]);
+  for (; r < r1; r += 32) add_bf16x8(acc, qh[static_cast<size_t>(r) * 8 + sub]);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
@@ -100,7 +113,7 @@ __global__ void __launch_bounds__(256) probe_partial_kernel(const uint16_t* __re
   if (threadIdx.x < kD) {
     double t = 0.0;
     for (int w = 0; w < 8; ++w) t += wsum[w][threadIdx.x];
-    partial[(static_cast<size_t>(hp) * gridDim.x + blockIdx.x) * kD + threadIdx.x] = t;
+    partial[(static_cast<size_t>(hp) * gridDim.x + blockIdx.x) * kD + threadIdx.x] = t * kBf16Unscale;
   }
 }
 
@@ -125,45 +138,80 @@ __global__ void __launch_bounds__(256) probe_mean_kernel(const double* __restric
 }
 
 // score_j = qbar . k_j / 8 (fp64 dot, fp32 result); special keys get -inf so they are never ranked.
-// Eight lanes per key row, each with one 16-byte chunk (a warp reads 4 whole rows, 512 contiguous
-// bytes, per load), two rows per lane group in flight; the 8 partial dots meet in 3 shuffles.
+// Each block takes a contiguous range of key rows.  Eight lanes per key row, each with one 16-byte
+// chunk (a warp reads 4 whole rows, 512 contiguous bytes, per load), kProbeRowsInFlight rows per
+// lane group loaded before any is used; the 8 partial dots of a row meet in 3 shuffles.  All lanes
+// of a warp take the same iterations (row validity is a per-group guard), so every shuffle has
+// its whole warp.
 __global__ void __launch_bounds__(256) probe_score_kernel(const uint16_t* __restrict__ k, int N, int V, int ns,
                                                           ProbeArgs a, const float* __restrict__ qbar,
                                                           float* __restrict__ scores) {
   const int hp = blockIdx.y;
   const int h = a.heads[hp];
-  const int sub = threadIdx.x & 7;
-  double qv[8];
+  const int sub = threadIdx.x & 7, grp = threadIdx.x >> 3;  // 32 row groups per block
+  double qv[8];  // this lane's 8 features of qbar, scaled by 2^896 against the 2^-896 of the keys
 #pragma unroll
-  for (int i = 0; i < 8; ++i) qv[i] = static_cast<double>(qbar[hp * kD + 8 * sub + i]);
+  for (int i = 0; i < 8; ++i) qv[i] = static_cast<double>(qbar[hp * kD + 8 * sub + i]) * kBf16Unscale;
   const uint4* kh = reinterpret_cast<const uint4*>(k + static_cast<size_t>(h) * N * kD);
-  const int groups = (gridDim.x * blockDim.x) >> 3;
-  for (int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 3; j < N; j += 2 * groups) {
-    const int j1 = j + groups;
-    const bool two = j1 < N;  // uniform over the 8 lanes of a row group
-    const uint4 w0 = kh[static_cast<size_t>(j) * 8 + sub];
-    const uint4 w1 = two ? kh[static_cast<size_t>(j1) * 8 + sub] : make_uint4(0u, 0u, 0u, 0u);
-    double x[8], d0 = 0.0, d1 = 0.0;
-    bf16x8_to_f64(w0, x);
+  float* sc = scores + static_cast<size_t>(hp) * N;
+  const int rows_per = (N + gridDim.x - 1) / gridDim.x;
+  const int r0 = blockIdx.x * rows_per, r1 = min(N, r0 + rows_per);
+  for (int jb = r0; jb < r1; jb += 32 * kProbeRowsInFlight) {
+    uint4 w[kProbeRowsInFlight];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) d0 = fma(qv[i], x[i], d0);
-    bf16x8_to_f64(w1, x);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) d1 = fma(qv[i], x[i], d1);
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      d0 += __shfl_xor_sync(0xffffffffu, d0, o);
-      d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+    for (int f = 0; f < kProbeRowsInFlight; ++f) {
+      const int jf = jb + 32 * f + grp;  // uniform over the 8 lanes of a row group
+      w[f] = jf < r1 ? kh[static_cast<size_t>(jf) * 8 + sub] : make_uint4(0u, 0u, 0u, 0u);
     }
+    double d[kProbeRowsInFlight];
+#pragma unroll
+    for (int f = 0; f < kProbeRowsInFlight; ++f) {
+      double x[8];
+      bf16x8_to_f64(w[f], x);
+      d[f] = 0.0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[f] = fma(qv[i], x[i], d[f]);
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+      for (int f = 0; f < kProbeRowsInFlight; ++f) d[f] += __shfl_xor_sync(0xffffffffu, d[f], o);
     if (sub == 0) {
-      scores[static_cast<size_t>(hp) * N + j] = (j % V) < ns ? -INFINITY : static_cast<float>(d0 * 0.125);
-      if (two) scores[static_cast<size_t>(hp) * N + j1] = (j1 % V) < ns ? -INFINITY : static_cast<float>(d1 * 0.125);
+#pragma unroll
+      for (int f = 0; f < kProbeRowsInFlight; ++f) {
+        const int jf = jb + 32 * f + grp;
+        if (jf < r1) sc[jf] = (jf % V) < ns ? -INFINITY : static_cast<float>(d[f] * 0.125);
+      }
     }
   }
 }
 
-// Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
-__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp /*[32]*/, int& total) {
+// ---- probe Top-K: a radix select spread over many blocks per head.
+//
+// The k-th largest order key is found one digit at a time (bits 31..21, 20..10, 9..0): every block
+// histograms the digit of the keys that match the digits chosen so far, adds its histogram into
+// the head's global one, and the last block to finish (a counter, no waiting) picks the digit
+// holding the k-th key and how many keys of equal prefix are still to be taken.  Then every block
+// counts, in its own contiguous chunk of keys, those above the final key and those equal to it,
+// and writes its selected indices in ascending order at the offset the counts of the chunks
+// before it give: all keys above the k-th, and the lowest-index keys equal to it.
+constexpr int kRankBins = 2048;   // 11-bit digits
+constexpr int kRankChunk = 4096;  // keys per block (256 threads x 16)
+constexpr int kRankPasses = 3;
+
+struct RankState {
+  uint32_t prefix;  // digits chosen so far
+  uint32_t mask;    // bits they cover
+  int remaining;    // keys still to take among those matching prefix under mask
+  int pad;
+};
+
+__host__ __device__ constexpr int rank_shift(int pass) { return pass == 0 ? 21 : (pass == 1 ? 10 : 0); }
+__host__ __device__ constexpr uint32_t rank_digit_mask(int pass) { return pass == 2 ? 0x3FFu : 0x7FFu; }
+
+// Exclusive scan of one int per thread over a block of kWarps warps; `total` gets the sum.
+template <int kWarps>
+__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp /*[kWarps]*/, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -174,89 +222,179 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* tmp /*[32]*/, in
   if (lane == 31) tmp[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = tmp[lane];
+    int w = lane < kWarps ? tmp[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    tmp[lane] = w;
+    if (lane < kWarps) tmp[lane] = w;
   }
   __syncthreads();
-  total = tmp[31];
+  total = tmp[kWarps - 1];
   const int before = warp > 0 ? tmp[warp - 1] : 0;
   __syncthreads();
   return before + x - v;
 }
 
-// Top-k of one probe head's scores: radix select of the k-th largest key, then an
-// ordered compaction that keeps every key above it and the lowest-index keys equal to it.
-__global__ void __launch_bounds__(1024) probe_topk_kernel(const float* __restrict__ scores, int N, ProbeArgs a,
-                                                          int32_t* __restrict__ cache) {
-  const int hp = blockIdx.x;
-  const int K = a.k[hp];
+// One digit pass over all keys of every probe head (grid: blocks per head x probe heads).
+// hist [n_probe][kRankPasses][kRankBins] and done [n_probe][kRankPasses] start at zero.
+__global__ void __launch_bounds__(256) probe_digit_kernel(const float* __restrict__ scores, int N, ProbeArgs a,
+                                                          int pass, int* __restrict__ hist,
+                                                          unsigned* __restrict__ done, RankState* __restrict__ st) {
+  const int hp = blockIdx.y;
   const float* sc = scores + static_cast<size_t>(hp) * N;
-  int32_t* out = cache + a.cache_off[hp];
-  __shared__ int hist[256];
-  __shared__ int tmp[32];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_remaining;
-
+  __shared__ int h[kRankBins];
+  __shared__ int tmp[8];
+  __shared__ bool last;
+  for (int i = threadIdx.x; i < kRankBins; i += blockDim.x) h[i] = 0;
   uint32_t prefix = 0, mask = 0;
-  int remaining = K;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < N; j += blockDim.x) {
-      const uint32_t key = order_key(sc[j]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int above = 0, b = 255;
-      for (; b > 0; --b) {
-        if (above + hist[b] >= remaining) break;
-        above += hist[b];
-      }
-      s_prefix = prefix | (static_cast<uint32_t>(b) << shift);
-      s_remaining = remaining - above;
-    }
-    __syncthreads();
-    prefix = s_prefix;
-    remaining = s_remaining;
-    mask |= 0xFFu << shift;
-    __syncthreads();
+  int remaining = a.k[hp];
+  if (pass > 0) {
+    const RankState r = st[hp];  // written by the previous pass's launch
+    prefix = r.prefix;
+    mask = r.mask;
+    remaining = r.remaining;
   }
-  // prefix is the k-th largest key; `remaining` keys equal to it are kept (lowest indices first).
-  const int per = (N + blockDim.x - 1) / blockDim.x;
-  const int j0 = threadIdx.x * per, j1 = min(N, j0 + per);
+  const int shift = rank_shift(pass);
+  const uint32_t dmask = rank_digit_mask(pass);
+  __syncthreads();
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < N; j += gridDim.x * blockDim.x) {
+    const uint32_t key = order_key(sc[j]);
+    if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & dmask], 1);
+  }
+  __syncthreads();
+  int* gh = hist + (static_cast<size_t>(hp) * kRankPasses + pass) * kRankBins;
+  for (int i = threadIdx.x; i < kRankBins; i += blockDim.x)
+    if (h[i] != 0) atomicAdd(&gh[i], h[i]);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&done[hp * kRankPasses + pass], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // the last block: thread t holds bins 2047-8t .. 2040-8t (descending), so a scan in thread
+  // order counts the keys above each bin
+  constexpr int kPer = kRankBins / 256;
+  int c[kPer], local = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    c[i] = __ldcg(&gh[kRankBins - 1 - kPer * threadIdx.x - i]);
+    local += c[i];
+  }
+  int total;
+  int above = block_exclusive_scan<8>(local, tmp, total);
+  const bool lowest = threadIdx.x == blockDim.x - 1;
+  if (above < remaining && (above + local >= remaining || lowest)) {
+    int bin = kRankBins - 1 - kPer * threadIdx.x;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      bin = kRankBins - 1 - kPer * static_cast<int>(threadIdx.x) - i;
+      if (above + c[i] >= remaining || bin == 0) break;
+      above += c[i];
+    }
+    RankState r;
+    r.prefix = prefix | (static_cast<uint32_t>(bin) << shift);
+    r.mask = mask | (dmask << shift);
+    r.remaining = remaining - above;
+    r.pad = 0;
+    st[hp] = r;
+  }
+}
+
+// Keys above the k-th key and keys equal to it in each block's chunk: counts [n_probe][blocks][2].
+__global__ void __launch_bounds__(256) probe_count_kernel(const float* __restrict__ scores, int N,
+                                                          const RankState* __restrict__ st,
+                                                          int* __restrict__ counts) {
+  const int hp = blockIdx.y;
+  const float* sc = scores + static_cast<size_t>(hp) * N;
+  const uint32_t kth = st[hp].prefix;
+  const int j0 = blockIdx.x * kRankChunk, j1 = min(N, j0 + kRankChunk);
+  int gt = 0, eq = 0;
+  for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+    const uint32_t key = order_key(sc[j]);
+    gt += key > kth;
+    eq += key == kth;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+  }
+  __shared__ int wg[8], we[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    wg[warp] = gt;
+    we[warp] = eq;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tg = 0, te = 0;
+    for (int w = 0; w < 8; ++w) {
+      tg += wg[w];
+      te += we[w];
+    }
+    counts[(static_cast<size_t>(hp) * gridDim.x + blockIdx.x) * 2] = tg;
+    counts[(static_cast<size_t>(hp) * gridDim.x + blockIdx.x) * 2 + 1] = te;
+  }
+}
+
+// The selected indices of each block's chunk, ascending, at the offset of the chunks before it.
+__global__ void __launch_bounds__(256) probe_write_kernel(const float* __restrict__ scores, int N, ProbeArgs a,
+                                                          const RankState* __restrict__ st,
+                                                          const int* __restrict__ counts,
+                                                          int32_t* __restrict__ cache) {
+  const int hp = blockIdx.y;
+  const float* sc = scores + static_cast<size_t>(hp) * N;
+  const uint32_t kth = st[hp].prefix;
+  const int remaining = st[hp].remaining;
+  __shared__ int tmp[8];
+  // keys above / equal in the chunks before this one
+  int gb = 0, eb = 0;
+  for (int b = threadIdx.x; b < static_cast<int>(blockIdx.x); b += blockDim.x) {
+    gb += counts[(static_cast<size_t>(hp) * gridDim.x + b) * 2];
+    eb += counts[(static_cast<size_t>(hp) * gridDim.x + b) * 2 + 1];
+  }
+  int gt_before, eq_before;
+  block_exclusive_scan<8>(gb, tmp, gt_before);
+  block_exclusive_scan<8>(eb, tmp, eq_before);
+  const int eq_chunk = max(0, remaining - eq_before);  // equal keys this chunk may still take
+  int32_t* out = cache + a.cache_off[hp] + gt_before + min(eq_before, remaining);
+  // each thread a contiguous run of the chunk, so the scans keep index order
+  constexpr int kRun = kRankChunk / 256;
+  const int j0 = blockIdx.x * kRankChunk + threadIdx.x * kRun, j1 = min(N, j0 + kRun);
+  uint32_t keys[kRun];
   int n_gt = 0, n_eq = 0;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t key = order_key(sc[j]);
-    n_gt += key > prefix;
-    n_eq += key == prefix;
+#pragma unroll
+  for (int i = 0; i < kRun; ++i) {
+    keys[i] = j0 + i < j1 ? order_key(sc[j0 + i]) : 0u;
+    n_gt += j0 + i < j1 && keys[i] > kth;
+    n_eq += j0 + i < j1 && keys[i] == kth;
   }
-  int tot_eq = 0, tot_gt = 0;
-  const int eq_before = block_exclusive_scan(n_eq, tmp, tot_eq);
-  const int eq_take = max(0, min(n_eq, remaining - eq_before));
-  const int mine = n_gt + eq_take;
-  const int pos0 = block_exclusive_scan(mine, tmp, tot_gt);
-  int pos = pos0, eq_seen = 0;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t key = order_key(sc[j]);
-    bool take = key > prefix;
-    if (key == prefix) {
+  int tot;
+  const int eq_mine_before = block_exclusive_scan<8>(n_eq, tmp, tot);
+  const int eq_take = max(0, min(n_eq, eq_chunk - eq_mine_before));
+  int pos = block_exclusive_scan<8>(n_gt + eq_take, tmp, tot);
+  int eq_seen = 0;
+#pragma unroll
+  for (int i = 0; i < kRun; ++i) {
+    if (j0 + i >= j1) break;
+    bool take = keys[i] > kth;
+    if (keys[i] == kth) {
       take = eq_seen < eq_take;
       ++eq_seen;
     }
-    if (take) out[pos++] = j;
+    if (take) out[pos++] = j0 + i;
   }
 }
 
 // Mean of L2-normalised DINO features over the patch tokens of each 64-token tile,
 // then normalised to unit length (its cosine against other tiles is a plain dot).
+// kChunks 16-byte chunks of a feature row per lane: dim <= 128 * kChunks.
+template <int kChunks>
 __global__ void __launch_bounds__(128) dino_pool_kernel(const float* __restrict__ dino, int N, int V, int ns,
-                                                        int P, int dim, float* __restrict__ tilevec) {
+                                                        int P, int dim, float* __restrict__ tilevec,
+                                                        __half* __restrict__ tile16, int dim16) {
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   extern __shared__ float pool_smem[];  // [4][dim] per-warp sums, then [dim] mean
@@ -265,34 +403,53 @@ __global__ void __launch_bounds__(128) dino_pool_kernel(const float* __restrict_
   __syncthreads();
   int count = 0;
   const int tok0 = t * kTile, tok1 = min(N, tok0 + kTile);
-  const int nc = dim >> 2;  // 16-byte chunks per feature row (dim is a multiple of 4, at most 1024)
-  for (int tok = tok0 + warp; tok < tok1; tok += 4) {
-    const int s = tok / V, loc = tok - s * V;
-    if (loc < ns) continue;
-    // the row once, in 16-byte loads, kept in registers for both passes
-    const float4* f = reinterpret_cast<const float4*>(dino + (static_cast<size_t>(s) * P + (loc - ns)) * dim);
-    float4 x[8];
-    float ss = 0.f;
+  const int nc = dim >> 2;  // 16-byte chunks per feature row (dim is a multiple of 4)
+  // four token rows per warp in flight: each lane loads its chunks of all four, then the four
+  // norms are reduced together and the normalised rows added to the warp's sums
+  constexpr int kRows = 4;
+  for (int tb = tok0 + warp * kRows; tb < tok1; tb += 4 * kRows) {
+    float4 x[kRows][kChunks];
+    float ss[kRows];
+    bool patch[kRows];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int i = 32 * c + lane;
-      x[c] = i < nc ? f[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-      ss = fmaf(x[c].x, x[c].x, fmaf(x[c].y, x[c].y, fmaf(x[c].z, x[c].z, fmaf(x[c].w, x[c].w, ss))));
+    for (int r = 0; r < kRows; ++r) {
+      const int tok = tb + r;
+      const int s = tok / V, loc = tok - s * V;
+      patch[r] = tok < tok1 && loc >= ns;
+      const float4* f = reinterpret_cast<const float4*>(dino + (static_cast<size_t>(s) * P + (loc - ns)) * dim);
+      ss[r] = 0.f;
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        const int i = 32 * c + lane;
+        x[r][c] = (patch[r] && i < nc) ? f[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float inv = 1.f / sqrtf(ss);
+    for (int r = 0; r < kRows; ++r)
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c)
+        ss[r] = fmaf(x[r][c].x, x[r][c].x,
+                     fmaf(x[r][c].y, x[r][c].y, fmaf(x[r][c].z, x[r][c].z, fmaf(x[r][c].w, x[r][c].w, ss[r]))));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], o);
     float4* w4 = reinterpret_cast<float4*>(wsum + warp * dim);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < kChunks; ++c) {
       const int i = 32 * c + lane;
       if (i < nc) {
-        float4 a = w4[i];
-        a.x += x[c].x * inv;
-        a.y += x[c].y * inv;
-        a.z += x[c].z * inv;
-        a.w += x[c].w * inv;
-        w4[i] = a;
+        float4 acc = w4[i];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          // a special token or a token past the tile contributes nothing
+          const float inv = patch[r] ? 1.f / sqrtf(ss[r]) : 0.f;
+          acc.x += x[r][c].x * inv;
+          acc.y += x[r][c].y * inv;
+          acc.z += x[r][c].z * inv;
+          acc.w += x[r][c].w * inv;
+        }
+        w4[i] = acc;
       }
     }
   }
@@ -311,6 +468,11 @@ __global__ void __launch_bounds__(128) dino_pool_kernel(const float* __restrict_
   __syncthreads();
   const float inv = 1.f / sqrtf(red[0] + red[1] + red[2] + red[3]);
   for (int c = threadIdx.x; c < dim; c += blockDim.x) tilevec[static_cast<size_t>(t) * dim + c] = mean[c] * inv;
+  if (tile16 != nullptr) {
+    // the same unit vector rounded to fp16, zero-padded to dim16 features (tensor-core operand)
+    for (int c = threadIdx.x; c < dim16; c += blockDim.x)
+      tile16[static_cast<size_t>(t) * dim16 + c] = __float2half_rn(c < dim ? mean[c] * inv : 0.f);
+  }
 }
 
 // Inverse of order_key.
@@ -359,9 +521,10 @@ __device__ __forceinline__ void warp_radix_kth(const float* row, int T, int kmax
 }
 
 // The kmax largest values of row[0..T) (ties to the lower index) written to out[0..kmax) in
-// rank order (value descending, then index ascending).  One warp.
+// rank order (value descending, then index ascending), as indices into row, or as map[index]
+// when a map is given.  One warp.
 __device__ __forceinline__ void warp_rank_row(const float* row, int T, int kmax, int* wh, int* widx, uint32_t* wkey,
-                                              int lane, int32_t* __restrict__ out) {
+                                              int lane, int32_t* __restrict__ out, const int* map = nullptr) {
   uint32_t prefix;
   int remaining;
   warp_radix_kth(row, T, kmax, wh, lane, prefix, remaining);
@@ -398,7 +561,7 @@ __device__ __forceinline__ void warp_rank_row(const float* row, int T, int kmax,
       const uint32_t kj = wkey[j];
       rank += (kj > ki) || (kj == ki && widx[j] < vi);
     }
-    out[rank] = vi;
+    out[rank] = map != nullptr ? map[vi] : vi;
   }
   __syncwarp();
 }
@@ -446,148 +609,10 @@ __global__ void __launch_bounds__(256) tile_topk_kernel(const float* __restrict_
                   sel_key + warp * kmax, lane, ranked + static_cast<size_t>(u0 + r) * kmax);
 }
 
-// Fast form for dim <= 384 (kTkChunks float4 chunks of 128 features per lane).
-//
-// Eight query tiles per block, one per warp for the ranking.  Every lane keeps its slice of
-// the eight query vectors in registers; a warp takes one candidate tile v at a time with
-// coalesced loads, forms eight fp32 partial dots and folds them over the warp with a
-// transposing butterfly (after it, lane group (lane>>2)&7 holds row r's full dot).
-//
-// fp32 accumulation misses the fp64 dot by at most (12 + 5) * 2^-24 * sum|a_i b_i| <= 1.02e-6
-// (unit vectors: sum|a_i b_i| <= 1; 12 products per lane, 5 butterfly levels).  So every tile
-// of the exact top-kmax has an fp32 cosine >= (the fp32 kmax-th value) - 2.04e-6, and every
-// tile below (the fp32 kmax-th value) - kTkBand cannot reach it.  The ranking therefore
-// recomputes exactly (fp64 dot, rounded to fp32 as the general form does) every tile within
-// kTkBand of the fp32 kmax-th value, and ranks the row: the result is the general form's.
-constexpr int kTkRows = 8;
+// Lane slices of the exact fp64 dots: kTkChunks float4 chunks of 128 features (dim <= 384).
 constexpr int kTkChunks = 3;
-constexpr float kTkBand = 4e-6f;
 
 __device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-
-// This lane's slice of kTkRows unit vectors (rows u0.. of `vec`; absent rows and features are 0).
-__device__ __forceinline__ void load_row_slices(const float* __restrict__ vec, int u0, int nr, int dim, int lane,
-                                                float4 (&q)[kTkRows][kTkChunks]) {
-#pragma unroll
-  for (int r = 0; r < kTkRows; ++r)
-#pragma unroll
-    for (int c = 0; c < kTkChunks; ++c) {
-      const int d = 128 * c + 4 * lane;
-      q[r][c] = (r < nr && d < dim) ? ld_f4(vec + static_cast<size_t>(u0 + r) * dim + d)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-}
-
-// fp32 dots of the kTkRows query vectors with candidates cand[0..n) (unit vectors, row-major,
-// `dim` wide) into cs[r * ld + v]: each warp takes one candidate at a time with coalesced loads
-// and folds its eight partial dots over the warp with a transposing butterfly (after it, lane
-// group (lane>>2)&7 holds row r's full dot).  All warps of the block take part.
-__device__ __forceinline__ void dots_fp32(const float4 (&q)[kTkRows][kTkChunks], const float* __restrict__ cand,
-                                          int n, int dim, int nr, float* cs, int ld, int warp, int lane) {
-  const int b2 = (lane >> 2) & 1, b3 = (lane >> 3) & 1, b4 = (lane >> 4) & 1;
-  const int my_row = (lane >> 2) & 7;
-  for (int v = warp; v < n; v += 8) {
-    const float* fv = cand + static_cast<size_t>(v) * dim;
-    float a[kTkRows];
-#pragma unroll
-    for (int r = 0; r < kTkRows; ++r) a[r] = 0.f;
-#pragma unroll
-    for (int c = 0; c < kTkChunks; ++c) {
-      const int d = 128 * c + 4 * lane;
-      if (d < dim) {
-        const float4 b = ld_f4(fv + d);
-#pragma unroll
-        for (int r = 0; r < kTkRows; ++r) {
-          a[r] = fmaf(q[r][c].x, b.x, a[r]);
-          a[r] = fmaf(q[r][c].y, b.y, a[r]);
-          a[r] = fmaf(q[r][c].z, b.z, a[r]);
-          a[r] = fmaf(q[r][c].w, b.w, a[r]);
-        }
-      }
-    }
-    float h4[4], h2[2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float send = b4 ? a[i] : a[i + 4], keep = b4 ? a[i + 4] : a[i];
-      h4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float send = b3 ? h4[i] : h4[i + 2], keep = b3 ? h4[i + 2] : h4[i];
-      h2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    float h1;
-    {
-      const float send = b2 ? h2[0] : h2[1], keep = b2 ? h2[1] : h2[0];
-      h1 = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
-    h1 += __shfl_xor_sync(0xffffffffu, h1, 1);
-    if ((lane & 3) == 0 && my_row < nr) cs[static_cast<size_t>(my_row) * ld + v] = h1;
-  }
-}
-
-// One warp: rank row[0..n) (fp32 dots of query row `rq` with candidates cand[0..n)) exactly.
-// Every candidate within kTkBand of the fp32 kmax-th value gets its exact value (fp64 dot,
-// rounded to fp32), then the row is ranked; out[0..kmax) receives candidate indices.
-__device__ __forceinline__ void rank_row_exact(float* row, int n, int kmax, const float4 (&q)[kTkRows][kTkChunks],
-                                               int rq, const float* __restrict__ cand, int dim, int* wh, int* widx,
-                                               uint32_t* wkey, int lane, int32_t* __restrict__ out) {
-  uint32_t prefix;
-  int remaining;
-  warp_radix_kth(row, n, kmax, wh, lane, prefix, remaining);
-  const float thr = key_value(prefix) - kTkBand;
-  for (int v0 = 0; v0 < n; v0 += 32) {
-    const int v = v0 + lane;
-    uint32_t todo = __ballot_sync(0xffffffffu, v < n && row[v] >= thr);
-    while (todo) {
-      const int bit = __ffs(todo) - 1;
-      todo &= todo - 1;
-      const int w = v0 + bit;
-      const float* fv = cand + static_cast<size_t>(w) * dim;
-      double acc = 0.0;
-#pragma unroll
-      for (int c = 0; c < kTkChunks; ++c) {
-        const int d = 128 * c + 4 * lane;
-        if (d < dim) {
-          const float4 b = ld_f4(fv + d);
-          float4 qa = q[0][c];
-#pragma unroll
-          for (int r = 1; r < kTkRows; ++r)
-            if (r == rq) qa = q[r][c];
-          acc = fma(static_cast<double>(qa.x), static_cast<double>(b.x), acc);
-          acc = fma(static_cast<double>(qa.y), static_cast<double>(b.y), acc);
-          acc = fma(static_cast<double>(qa.z), static_cast<double>(b.z), acc);
-          acc = fma(static_cast<double>(qa.w), static_cast<double>(b.w), acc);
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) row[w] = static_cast<float>(acc);
-    }
-  }
-  __syncwarp();
-  warp_rank_row(row, n, kmax, wh, widx, wkey, lane, out);
-}
-
-__global__ void __launch_bounds__(256) tile_topk_fast_kernel(const float* __restrict__ tilevec, int T, int dim,
-                                                             int kmax, int32_t* __restrict__ ranked) {
-  extern __shared__ uint8_t tk_smem[];
-  float* cs = reinterpret_cast<float*>(tk_smem);                               // [8][T]
-  int* hist = reinterpret_cast<int*>(cs + static_cast<size_t>(kTkRows) * T);  // [8 warps][256]
-  int* sel_idx = hist + 8 * 256;                                               // [8 warps][kmax]
-  uint32_t* sel_key = reinterpret_cast<uint32_t*>(sel_idx + 8 * kmax);         // [8 warps][kmax]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u0 = blockIdx.x * kTkRows;
-  const int nr = min(kTkRows, T - u0);
-  float4 q[kTkRows][kTkChunks];
-  load_row_slices(tilevec, u0, nr, dim, lane, q);
-  dots_fp32(q, tilevec, T, dim, nr, cs, T, warp, lane);
-  __syncthreads();
-  if (warp >= nr) return;
-  rank_row_exact(cs + static_cast<size_t>(warp) * T, T, kmax, q, warp, tilevec, dim, hist + warp * 256,
-                 sel_idx + warp * kmax, sel_key + warp * kmax, lane, ranked + static_cast<size_t>(u0 + warp) * kmax);
-}
 
 // ---- token-wise DINO Top-K (section 4.1, "DINO Top-K Kernel": per query token, the Top-K most
 // similar tokens of every frame; section 5.1: K per frame)
@@ -939,6 +964,125 @@ __global__ void __launch_bounds__(256, 3) token_rank_kernel(const __half* __rest
 constexpr int kGroupWindow = 64;
 constexpr int kMaxSortTiles = 16384;
 
+// ---- block-wise DINO Top-K ranking (section 4.3, "DINO Top-K Kernel", block-wise variant)
+//
+// The cosines of a chunk of query tiles against all T tiles come from the tensor cores (the tile
+// unit vectors rounded to fp16, token_sim.cu: within kTokScoreErr of the exact cosine).  One warp
+// per query tile u ranks its row.  With A_k the kmax-th largest approximate cosine, every tile of
+// the exact Top-kmax has an approximate cosine >= A_k - 2 kTokScoreErr, and every tile below that
+// has an exact value below all of theirs (the argument above token_rank_frame).  Those candidates
+// get their exact value (fp64 dot of the fp32 unit vectors, rounded to fp32) and are ranked by it,
+// value descending, ties to the lower tile index: the row's exact ranking.  Up to kTrCap
+// candidates are listed in index order and recomputed four at a time; a row with more (many
+// near-equal cosines) is recomputed in place, one candidate at a time.
+constexpr int kTrCap = 256;
+
+__host__ __device__ inline size_t tile_rank_warp_bytes(int T, int kmax) {
+  const size_t row = (sizeof(float) * static_cast<size_t>(T) + 15) & ~size_t(15);
+  return row + (sizeof(int) + sizeof(float)) * kTrCap + sizeof(int) * 256 +
+         ((3 * sizeof(int) * static_cast<size_t>(kmax) + 15) & ~size_t(15));
+}
+
+// fp64 dots of the lane slices q with candidate rows idx[0..kN) (idx[j] for j >= n repeats
+// idx[0]), all kN rows' loads in flight together, each summed over the warp.
+template <int kN>
+__device__ __forceinline__ void exact_dots(const float4 (&q)[kTkChunks], const float* __restrict__ cand,
+                                           const int* idx, int n, int dim, int lane, double (&e)[kN]) {
+  float4 b[kN][kTkChunks];
+#pragma unroll
+  for (int j = 0; j < kN; ++j) {
+    const float* f = cand + static_cast<size_t>(idx[j < n ? j : 0]) * dim;
+#pragma unroll
+    for (int c = 0; c < kTkChunks; ++c) {
+      const int d = 128 * c + 4 * lane;
+      b[j][c] = d < dim ? ld_f4(f + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kN; ++j) e[j] = 0.0;
+#pragma unroll
+  for (int c = 0; c < kTkChunks; ++c) {
+    const double qx = q[c].x, qy = q[c].y, qz = q[c].z, qw = q[c].w;
+#pragma unroll
+    for (int j = 0; j < kN; ++j) {
+      e[j] = fma(qx, static_cast<double>(b[j][c].x), e[j]);
+      e[j] = fma(qy, static_cast<double>(b[j][c].y), e[j]);
+      e[j] = fma(qz, static_cast<double>(b[j][c].z), e[j]);
+      e[j] = fma(qw, static_cast<double>(b[j][c].w), e[j]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int j = 0; j < kN; ++j) e[j] += __shfl_xor_sync(0xffffffffu, e[j], o);
+}
+
+// Rows r0 .. r0 + rows of the ranked tile lists from the chunk's approximate cosines
+// scores[rows][ld] (fp16); blockDim.x / 32 warps, one query tile each.
+__global__ void __launch_bounds__(256) tile_rank_kernel(const __half* __restrict__ scores, long long ld, int r0,
+                                                        int rows, const float* __restrict__ tilevec, int T, int dim,
+                                                        int kmax, int32_t* __restrict__ ranked) {
+  extern __shared__ __align__(16) uint8_t tr_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lr = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (lr >= rows) return;  // no block-wide barrier below
+  uint8_t* w = tr_smem + static_cast<size_t>(warp) * tile_rank_warp_bytes(T, kmax);
+  float* row = reinterpret_cast<float*>(w);  // [T] approximate cosines
+  int* cl = reinterpret_cast<int*>(w + ((sizeof(float) * static_cast<size_t>(T) + 15) & ~size_t(15)));  // [kTrCap]
+  float* ev = reinterpret_cast<float*>(cl + kTrCap);   // [kTrCap] exact values of the listed candidates
+  int* hist = reinterpret_cast<int*>(ev + kTrCap);     // [256]
+  int* widx = hist + 256;                              // [kmax]
+  uint32_t* wkey = reinterpret_cast<uint32_t*>(widx + kmax);  // [kmax]
+  const int u = r0 + lr;
+  float4 q[kTkChunks];
+  load_one_slice(tilevec, u, dim, lane, q);
+  const __half* srow = scores + static_cast<size_t>(lr) * ld;
+  for (int v = lane; v < T; v += 32) row[v] = __half2float(srow[v]);
+  __syncwarp();
+  uint32_t prefix;
+  int remaining;
+  warp_radix_kth(row, T, kmax, hist, lane, prefix, remaining);
+  const float thr = key_value(prefix) - 2.f * kTokScoreErr;
+  int m = 0;
+  for (int v0 = 0; v0 < T; v0 += 32) {
+    const int v = v0 + lane;
+    const bool take = v < T && row[v] >= thr;
+    const uint32_t mask = __ballot_sync(0xffffffffu, take);
+    const int pos = m + __popc(mask & ((1u << lane) - 1u));
+    if (take && pos < kTrCap) cl[pos] = v;
+    m += __popc(mask);
+  }
+  __syncwarp();
+  int32_t* out = ranked + static_cast<size_t>(u) * kmax;
+  if (m <= kTrCap) {
+    for (int i = 0; i < m; i += 4) {
+      double e[4];
+      exact_dots<4>(q, tilevec, cl + i, m - i, dim, lane, e);
+      if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (i + j < m) ev[i + j] = static_cast<float>(e[j]);
+      }
+    }
+    __syncwarp();
+    warp_rank_row(ev, m, kmax, hist, widx, wkey, lane, out, cl);
+  } else {
+    // every other tile keeps its approximate value, below all exact Top-kmax values
+    for (int v0 = 0; v0 < T; v0 += 32) {
+      const int v = v0 + lane;
+      uint32_t todo = __ballot_sync(0xffffffffu, v < T && row[v] >= thr);
+      while (todo) {
+        const int bit = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const double e = exact_dot(q, tilevec + static_cast<size_t>(v0 + bit) * dim, dim, lane);
+        if (lane == 0) row[v0 + bit] = static_cast<float>(e);
+      }
+    }
+    __syncwarp();
+    warp_rank_row(row, T, kmax, hist, widx, wkey, lane, out);
+  }
+}
+
 __global__ void __launch_bounds__(1024) corr_sort_kernel(const int32_t* __restrict__ ranked, int T, int kmax,
                                                          int r, int32_t* __restrict__ order) {
   extern __shared__ unsigned long long keys[];  // [pow2 >= T]
@@ -1079,6 +1223,49 @@ TokWs token_ws(long long R, int dim) {
   return t;
 }
 
+// Correspondence part of the select workspace, offsets from its (256-byte aligned) start: fp32 tile
+// unit vectors [T][dim], grouping bitsets [T][words], sorted tiles [T]; with the tensor-core
+// cosines (dim <= 384) also fp16 tile unit vectors [T][dim16] (zero-padded to a multiple of 64
+// features) and the fp16 cosines of one chunk of query tiles [chunk_rows][ld] (ld = T rounded up
+// to 8; chunks of at most kTileScoreBudget bytes).
+constexpr size_t kTileScoreBudget = size_t(16) << 20;
+
+struct CorrWs {
+  bool tc;
+  int dim16, chunk_rows;
+  long long ld;
+  size_t tilevec, bits, sorted, tile16, scores, end;
+};
+
+CorrWs corr_ws(int T, int dim) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  CorrWs c;
+  c.tc = dim <= 128 * kTkChunks;
+  c.dim16 = (dim + 63) / 64 * 64;
+  c.ld = (static_cast<long long>(T) + 7) / 8 * 8;
+  long long rows = static_cast<long long>(kTileScoreBudget / (static_cast<size_t>(c.ld) * 2)) / 128 * 128;
+  if (rows < 128) rows = 128;
+  c.chunk_rows = static_cast<int>(rows < T ? rows : T);
+  c.tilevec = 0;
+  c.bits = al(static_cast<size_t>(T) * dim * sizeof(float));
+  c.sorted = al(c.bits + static_cast<size_t>(T) * ((T + 31) / 32) * sizeof(uint32_t));
+  c.end = al(c.sorted + static_cast<size_t>(T) * sizeof(int32_t));
+  c.tile16 = c.scores = c.end;
+  if (c.tc) {
+    c.scores = al(c.tile16 + static_cast<size_t>(T) * c.dim16 * 2);
+    c.end = al(c.scores + static_cast<size_t>(c.chunk_rows) * c.ld * 2);
+  }
+  return c;
+}
+
+// Probe Top-K scratch: digit histograms and pass counters (zeroed per build), per-chunk counts.
+size_t rank_zero_bytes(int n_probe) {
+  return static_cast<size_t>(n_probe) * kRankPasses * (kRankBins * sizeof(int) + sizeof(unsigned));
+}
+size_t rank_counts_bytes(int n_probe, int N) {
+  return static_cast<size_t>(n_probe) * ((N + kRankChunk - 1) / kRankChunk) * 2 * sizeof(int);
+}
+
 size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows) {
   size_t b = 0;
   b += static_cast<size_t>(n_probe) * kProbePartials * kD * sizeof(double);
@@ -1086,13 +1273,13 @@ size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, lon
   b = (b + 255) & ~size_t(255);
   b += static_cast<size_t>(n_probe) * N * sizeof(float);
   b = (b + 255) & ~size_t(255);
-  if (corr) {
-    b += static_cast<size_t>(T) * dim * sizeof(float);
-    b = (b + 255) & ~size_t(255);
-    b += static_cast<size_t>(T) * ((T + 31) / 32) * sizeof(uint32_t);  // grouping bitsets
-    b = (b + 255) & ~size_t(255);
-    b += static_cast<size_t>(T) * sizeof(int32_t);                      // sorted tiles
-  }
+  b += rank_zero_bytes(n_probe);
+  b = (b + 255) & ~size_t(255);
+  b += static_cast<size_t>(n_probe) * sizeof(RankState);
+  b = (b + 255) & ~size_t(255);
+  b += rank_counts_bytes(n_probe, N);
+  b = (b + 255) & ~size_t(255);
+  if (corr) b += corr_ws(T, dim).end;
   b = ((b + 255) & ~size_t(255)) + 256;
   if (tok_rows > 0) b += token_ws(tok_rows, dim).end;
   return b;
@@ -1127,6 +1314,16 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
   float* scores = reinterpret_cast<float*>(ws + off);
   off += static_cast<size_t>(sp.n_probe) * sp.N * sizeof(float);
   off = (off + 255) & ~size_t(255);
+  int* rank_hist = reinterpret_cast<int*>(ws + off);  // zeroed with rank_done in one memset
+  unsigned* rank_done = reinterpret_cast<unsigned*>(rank_hist + static_cast<size_t>(sp.n_probe) * kRankPasses * kRankBins);
+  off += rank_zero_bytes(sp.n_probe);
+  off = (off + 255) & ~size_t(255);
+  RankState* rank_state = reinterpret_cast<RankState*>(ws + off);
+  off += static_cast<size_t>(sp.n_probe) * sizeof(RankState);
+  off = (off + 255) & ~size_t(255);
+  int* rank_counts = reinterpret_cast<int*>(ws + off);
+  off += rank_counts_bytes(sp.n_probe, sp.N);
+  off = (off + 255) & ~size_t(255);
   float* tilevec = reinterpret_cast<float*>(ws + off);
 
   if (sp.n_probe > 0) {
@@ -1139,25 +1336,64 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
     }
     probe_partial_kernel<<<dim3(kProbePartials, sp.n_probe), 256, 0, stream>>>(q, sp.N, a, partial);
     probe_mean_kernel<<<sp.n_probe, 4 * kD, 0, stream>>>(partial, kProbePartials, sp.N, qbar);
-    // 32 key rows per 256-thread block and step; at most 8 blocks per SM and head
-    const int score_blocks = std::max(1, std::min((sp.N + 63) / 64, 8 * sp.num_sms));
+    // contiguous ranges of key rows, 32 x kProbeRowsInFlight rows per block and step
+    const int score_blocks = std::max(1, std::min((sp.N + 127) / 128, 2 * sp.num_sms));
     probe_score_kernel<<<dim3(score_blocks, sp.n_probe), 256, 0, stream>>>(k, sp.N, sp.V, sp.ns, a, qbar, scores);
-    probe_topk_kernel<<<sp.n_probe, 1024, 0, stream>>>(scores, sp.N, a, cache);
-    *n_launch += 4;
+    const int rank_blocks = (sp.N + kRankChunk - 1) / kRankChunk;
+    cudaError_t e = cudaMemsetAsync(rank_hist, 0, rank_zero_bytes(sp.n_probe), stream);
+    if (e != cudaSuccess) return e;
+    for (int pass = 0; pass < kRankPasses; ++pass)
+      probe_digit_kernel<<<dim3(rank_blocks, sp.n_probe), 256, 0, stream>>>(scores, sp.N, a, pass, rank_hist,
+                                                                           rank_done, rank_state);
+    probe_count_kernel<<<dim3(rank_blocks, sp.n_probe), 256, 0, stream>>>(scores, sp.N, rank_state, rank_counts);
+    probe_write_kernel<<<dim3(rank_blocks, sp.n_probe), 256, 0, stream>>>(scores, sp.N, a, rank_state, rank_counts,
+                                                                         cache);
+    *n_launch += 3 + kRankPasses + 2;
   }
   if (sp.corr_kmax > 0) {
+    const CorrWs cw = corr_ws(sp.T, sp.dim);
+    uint8_t* cbase = reinterpret_cast<uint8_t*>(tilevec);
     const size_t pool_smem = sizeof(float) * 5 * sp.dim;
-    dino_pool_kernel<<<sp.T, 128, pool_smem, stream>>>(dino, sp.N, sp.V, sp.ns, sp.P, sp.dim, tilevec);
+    const size_t rank_warp = tile_rank_warp_bytes(sp.T, sp.corr_kmax);
+    const int rank_warps = static_cast<int>(std::min<size_t>(8, (112 * 1024) / rank_warp));
     cudaError_t e = cudaSuccess;
-    const size_t fast_smem = sizeof(float) * static_cast<size_t>(kTkRows) * sp.T +
-                             sizeof(int) * (8 * 256 + 16 * static_cast<size_t>(sp.corr_kmax));
-    if (sp.dim <= 128 * kTkChunks && fast_smem <= 200 * 1024) {
-      e = cudaFuncSetAttribute(tile_topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(fast_smem));
+    if (cw.tc && rank_warps >= 1) {
+      // cosines on the tensor cores (fp16 operands), exact ranking of the candidates they leave
+      __half* tile16 = reinterpret_cast<__half*>(cbase + cw.tile16);
+      __half* tscores = reinterpret_cast<__half*>(cbase + cw.scores);
+      dino_pool_kernel<3><<<sp.T, 128, pool_smem, stream>>>(dino, sp.N, sp.V, sp.ns, sp.P, sp.dim, tilevec, tile16,
+                                                            cw.dim16);
+      ++*n_launch;
+      CUtensorMap tm;
+      if (!make_map_f16_rows(&tm, tile16, sp.T, cw.dim16)) return cudaErrorInvalidValue;
+      const size_t rsmem = rank_warps * rank_warp;
+      e = cudaFuncSetAttribute(tile_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(rsmem));
       if (e != cudaSuccess) return e;
-      tile_topk_fast_kernel<<<(sp.T + kTkRows - 1) / kTkRows, 256, fast_smem, stream>>>(
-          tilevec, sp.T, sp.dim, sp.corr_kmax, cache + sp.corr_off);
+      for (int r0 = 0; r0 < sp.T; r0 += cw.chunk_rows) {
+        const int rows = std::min(cw.chunk_rows, sp.T - r0);
+        TokenSimParams tp;
+        tp.r0 = r0;
+        tp.rows = rows;
+        tp.n_rb = (rows + 127) / 128;
+        tp.n_ct = (sp.T + 255) / 256;
+        tp.n_kc = cw.dim16 / 64;
+        tp.ld = cw.ld;
+        tp.scores = reinterpret_cast<uint16_t*>(tscores);
+        tp.err = sp.err;
+        tp.wait_budget = sp.wait_budget;
+        e = launch_token_sim(tp, tm, sp.num_sms, stream);
+        if (e != cudaSuccess) return e;
+        tile_rank_kernel<<<(rows + rank_warps - 1) / rank_warps, 32 * rank_warps, rsmem, stream>>>(
+            tscores, cw.ld, r0, rows, tilevec, sp.T, sp.dim, sp.corr_kmax, cache + sp.corr_off);
+        *n_launch += 2;
+      }
     } else {
+      if (sp.dim <= 128 * 3)
+        dino_pool_kernel<3><<<sp.T, 128, pool_smem, stream>>>(dino, sp.N, sp.V, sp.ns, sp.P, sp.dim, tilevec,
+                                                              nullptr, 0);
+      else
+        dino_pool_kernel<8><<<sp.T, 128, pool_smem, stream>>>(dino, sp.N, sp.V, sp.ns, sp.P, sp.dim, tilevec,
+                                                              nullptr, 0);
       const int R = tile_rows_per_block(sp.T, sp.dim, sp.corr_kmax);
       if (R <= 0) return cudaErrorInvalidValue;
       const size_t smem = sizeof(float) * (static_cast<size_t>(R) * sp.dim + static_cast<size_t>(R) * sp.T) +
@@ -1166,17 +1402,12 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
       if (e != cudaSuccess) return e;
       tile_topk_kernel<<<(sp.T + R - 1) / R, 256, smem, stream>>>(tilevec, sp.T, sp.dim, R, sp.corr_kmax,
                                                                   cache + sp.corr_off);
+      *n_launch += 2;
     }
-    *n_launch += 2;
     // query-tile grouping for the attention work items
-    size_t goff = static_cast<size_t>(reinterpret_cast<uint8_t*>(tilevec) - ws) +
-                  static_cast<size_t>(sp.T) * sp.dim * sizeof(float);
-    goff = (goff + 255) & ~size_t(255);
     const int words = (sp.T + 31) / 32;
-    uint32_t* bits = reinterpret_cast<uint32_t*>(ws + goff);
-    goff += static_cast<size_t>(sp.T) * words * sizeof(uint32_t);
-    goff = (goff + 255) & ~size_t(255);
-    int32_t* sorted = reinterpret_cast<int32_t*>(ws + goff);
+    uint32_t* bits = reinterpret_cast<uint32_t*>(cbase + cw.bits);
+    int32_t* sorted = reinterpret_cast<int32_t*>(cbase + cw.sorted);
     int32_t* order = cache + sp.order_off;
     if (sp.T <= kMaxSortTiles) {
       int n2 = 1;

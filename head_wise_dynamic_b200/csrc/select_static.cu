@@ -1,11 +1,10 @@
 // saf3r_select_kv_static: the per-input index build without a caller workspace.
 //
 // saf3r_select_kv needs a device workspace for its partial sums, probe scores,
-// tile descriptors and grouping bitsets, and expects the caller to allocate it.
-// Some callers cannot: code that records work into a CUDA graph while a stream
-// is being captured (device allocation is not allowed there), engines whose
-// latency-critical loop must never enter an allocator, and plug-in hosts that
-// hand a library only its input and output buffers.  This entry point serves
+// tile descriptors, tile cosines and grouping bitsets, and expects the caller to
+// allocate it.  Some callers cannot: engines whose latency-critical loop must
+// never enter an allocator, and plug-in hosts that hand a library only its input
+// and output buffers.  This entry point serves
 // them from a fixed device array compiled into the library instead, so it calls
 // no allocator at all; the array costs every GPU that loads the library
 // kStaticScratchBytes of memory until the process exits.
@@ -20,8 +19,8 @@ namespace {
 
 // Largest select workspace this entry point can serve (saf3r_workspace_bytes with
 // SAF3R_OP_SELECT): enough for the 274,800-token layer with 4 probe heads and
-// 4 correspondence heads.
-constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+// 4 correspondence heads (32.3 MiB, most of it the fp16 tile cosines of one chunk).
+constexpr size_t kStaticScratchBytes = size_t(40) << 20;
 
 static __device__ __align__(256) unsigned char g_select_scratch[kStaticScratchBytes];
 

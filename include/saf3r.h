@@ -145,17 +145,18 @@ saf3r_status saf3r_select_kv(const saf3r_layout* layout, const saf3r_head_cfg* c
 /*
  * saf3r_select_kv without a caller workspace.  No counterpart in the paper: this
  * entry point exists for callers that cannot allocate device memory for the
- * workspace - work recorded into a CUDA graph while a stream is captured (device
- * allocation is not allowed there), engines whose latency-critical loop must not
- * enter an allocator, plug-in hosts that pass a library only its inputs and
- * outputs.  It builds exactly the cache saf3r_select_kv builds, taking its
- * scratch from a 16 MiB device array compiled into the library (held by every
- * GPU that loads the library until the process exits), and calls no allocator.
+ * workspace - engines whose latency-critical loop must not enter an allocator,
+ * plug-in hosts that pass a library only its inputs and outputs.  It builds
+ * exactly the cache saf3r_select_kv builds, taking its scratch from a 40 MiB
+ * device array compiled into the library (held by every GPU that loads the
+ * library until the process exits), and calls no allocator.
  *   - Limit: saf3r_workspace_bytes(layout, cfg, SAF3R_OP_SELECT) must be at most
- *     16 MiB (16777216 bytes); larger layers return SAF3R_ERR_UNSUPPORTED and
- *     launch nothing.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     40 MiB (41943040 bytes; the 274,800-token layer with 4 probe and 4
+ *     correspondence heads needs 32.3 MiB); larger layers return
+ *     SAF3R_ERR_UNSUPPORTED and launch nothing.
+ *   - First-call setup: the first call on each device looks up the array's
+ *     device address (cudaGetSymbolAddress) and remembers it; later calls on
+ *     that device reuse it.
  *   - All calls share the one array: calls that may overlap on the GPU (other
  *     streams, other host threads) race and must be serialised by the caller.
  *     Nothing in the array needs to start at zero; each call clears what it needs.

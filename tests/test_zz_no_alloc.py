@@ -1,7 +1,7 @@
 """The allocation-free index build, saf3r_select_kv_static, against saf3r_select_kv.
 
-Callers that cannot allocate device memory (stream capture into a CUDA graph,
-allocator-free latency loops, hosts that pass only inputs and outputs) use the
+Callers that cannot allocate device memory (allocator-free latency loops, hosts
+that pass only inputs and outputs) use the
 static entry point; it must build the same cache as the regular one.  This file
 is collected last so that a failure here comes after every other test ran."""
 import numpy as np
@@ -58,11 +58,11 @@ def test_static_select_matches_regular_on_two_calls(name):
 def test_static_select_rejects_layers_beyond_its_scratch():
     import head_wise_dynamic_b200 as hw
     from saf3r_synth import CORR, PROBE, HeadCfg, Layout
-    big = Layout(S=400, g=37, H=8)  # T = 8588 tiles: grouping bitsets alone exceed 9 MB
+    big = Layout(S=400, g=37, H=8)  # T = 8588 tiles: 51 MiB of select workspace
     heads = [HeadCfg(PROBE, k=1000)] * 4 + [HeadCfg(CORR, k=64)] * 4
     L = hw.layout_of(big)
     cfg = hw.cfg_array(heads)
-    assert hw.saf3r_workspace_bytes(L, cfg, hw.OP_SELECT) > 16 << 20
+    assert hw.saf3r_workspace_bytes(L, cfg, hw.OP_SELECT) > 40 << 20
     dummy = torch.empty(1024, dtype=torch.uint8, device="cuda")
     with pytest.raises(hw.Saf3rError) as e:
         hw.saf3r_select_kv_static(L, cfg, dummy, dummy, dummy, dummy)
