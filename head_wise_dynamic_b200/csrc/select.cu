@@ -20,7 +20,7 @@ namespace saf3r {
 
 namespace {
 
-constexpr int kProbePartials = 296;  // row blocks per probe head (2 x 148 SMs)
+constexpr int kProbePartials = 296;  // most row blocks (partial sums) per probe head
 #ifndef SAF3R_PROBE_ROWS_IN_FLIGHT
 #define SAF3R_PROBE_ROWS_IN_FLIGHT 4
 #endif
@@ -46,7 +46,15 @@ struct ProbeArgs {
 // products of such scaled values round exactly as those of the unscaled ones in the same order
 // (a power-of-two scale commutes with rounding while the result is normal; below that, every sum
 // of bf16 values is a multiple of 2^-133 and exact either way).
-constexpr double kBf16Unscale = 0x1p896;
+constexpr double kUnscale896 = 0x1p896;
+
+// fp32 -> fp64 the same way: the sign, 8-bit exponent and 23-bit mantissa placed in a double's
+// layout without rebiasing read as x * 2^-896 exactly (finite x, subnormals included).  Against an
+// operand pre-multiplied by 2^896 the products are the unscaled ones, rounded alike.
+__device__ __forceinline__ double f32_scaled(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return __hiloint2double(static_cast<int>((u & 0x80000000u) | ((u & 0x7FFFFFFFu) >> 3)), static_cast<int>(u << 29));
+}
 __device__ __forceinline__ double bf16_lo_scaled(uint32_t w) {
   return __hiloint2double(static_cast<int>(((w & 0x8000u) << 16) | ((w & 0x7FFFu) << 13)), 0);
 }
@@ -74,12 +82,16 @@ __device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4& w) {
   for (int i = 0; i < 8; ++i) acc[i] += x[i];
 }
 
-// Partial fp64 column sums of Q_h over a range of rows.  Lane l of a warp reads the 16-byte
-// chunk (l % 8) of row r + l / 8 (a warp reads 4 whole rows, 512 contiguous bytes, per load) and
-// keeps the 8 column sums of its chunk; kProbeRowsInFlight rows per lane are loaded before any is
-// added.  The lanes and warps that share a chunk are added in a fixed order at the end.
-__global__ void __launch_bounds__(256) probe_partial_kernel(const uint16_t* __restrict__ q, int N,
-                                                            ProbeArgs a, double* __restrict__ partial) {
+// qbar = (1/N) sum_i q_i for every probe head, in one launch.  Each block sums a contiguous
+// range of rows: lane l of a warp reads the 16-byte chunk (l % 8) of row r + l / 8 (a warp reads
+// 4 whole rows, 512 contiguous bytes, per load) and keeps the 8 column sums of its chunk; the
+// next step's kProbeRowsInFlight rows are requested before this step's are added.  The lanes
+// and warps that share a chunk are added in a fixed order into the block's partial sums; the
+// last block of a head to finish (a counter, no waiting) adds the head's partials in a fixed
+// order and rounds the mean once to fp32.  done[n_probe] starts at zero.
+__global__ void __launch_bounds__(256) probe_mean_kernel(const uint16_t* __restrict__ q, int N, ProbeArgs a,
+                                                         double* __restrict__ partial, unsigned* __restrict__ done,
+                                                         float* __restrict__ qbar) {
   const int hp = blockIdx.y;
   const int h = a.heads[hp];
   const int rows_per = (N + gridDim.x - 1) / gridDim.x;
@@ -87,60 +99,70 @@ __global__ void __launch_bounds__(256) probe_partial_kernel(const uint16_t* __re
   const int r1 = min(N, r0 + rows_per);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = lane & 7;
   const uint4* qh = reinterpret_cast<const uint4*>(q + static_cast<size_t>(h) * N * kD);
+  constexpr int kStep = 32 * kProbeRowsInFlight;
   double acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-  int r = r0 + warp * 4 + (lane >> 3);
-  for (; r + 32 * (kProbeRowsInFlight - 1) < r1; r += 32 * kProbeRowsInFlight) {
-    uint4 w[kProbeRowsInFlight];
+  const int rl = r0 + warp * 4 + (lane >> 3);  // this lane's first row
+  uint4 w[kProbeRowsInFlight];
 #pragma unroll
-    for (int f = 0; f < kProbeRowsInFlight; ++f) w[f] = qh[static_cast<size_t>(r + 32 * f) * 8 + sub];
-#pragma unroll
-    for (int f = 0; f < kProbeRowsInFlight; ++f) add_bf16x8(acc, w[f]);
+  for (int f = 0; f < kProbeRowsInFlight; ++f) {
+    const int r = rl + 32 * f;
+    w[f] = r < r1 ? qh[static_cast<size_t>(r) * 8 + sub] : make_uint4(0u, 0u, 0u, 0u);
   }
-  for (; r < r1; r += 32) add_bf16x8(acc, qh[static_cast<size_t>(r) * 8 + sub]);
+  for (int rb = rl; rb < r1; rb += kStep) {
+    uint4 nx[kProbeRowsInFlight];
+#pragma unroll
+    for (int f = 0; f < kProbeRowsInFlight; ++f) {
+      const int r = rb + kStep + 32 * f;
+      nx[f] = r < r1 ? qh[static_cast<size_t>(r) * 8 + sub] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int f = 0; f < kProbeRowsInFlight; ++f) add_bf16x8(acc, w[f]);  // rows past r1 add zeros
+#pragma unroll
+    for (int f = 0; f < kProbeRowsInFlight; ++f) w[f] = nx[f];
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 8);
     acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
   }
   __shared__ double wsum[8][kD];
+  __shared__ bool last;
   if (lane < 8) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) wsum[warp][8 * sub + i] = acc[i];
   }
   __syncthreads();
+  double* hpart = partial + static_cast<size_t>(hp) * gridDim.x * kD;
   if (threadIdx.x < kD) {
     double t = 0.0;
-    for (int w = 0; w < 8; ++w) t += wsum[w][threadIdx.x];
-    partial[(static_cast<size_t>(hp) * gridDim.x + blockIdx.x) * kD + threadIdx.x] = t * kBf16Unscale;
+    for (int w8 = 0; w8 < 8; ++w8) t += wsum[w8][threadIdx.x];
+    hpart[static_cast<size_t>(blockIdx.x) * kD + threadIdx.x] = t * kUnscale896;
   }
-}
-
-// qbar = (sum of partials) / N, rounded once to fp32.  Four threads per column take every
-// fourth partial; their sums are added in a fixed order.
-__global__ void __launch_bounds__(256) probe_mean_kernel(const double* __restrict__ partial, int nparts, int N,
-                                                         float* __restrict__ qbar) {
-  const int hp = blockIdx.x, c = threadIdx.x & (kD - 1), g = threadIdx.x >> 6;
-  const double* base = partial + static_cast<size_t>(hp) * nparts * kD + c;
-  double t0 = 0.0, t1 = 0.0;
-  int b = g;
-  for (; b + 4 < nparts; b += 8) {
-    t0 += base[static_cast<size_t>(b) * kD];
-    t1 += base[static_cast<size_t>(b + 4) * kD];
-  }
-  if (b < nparts) t0 += base[static_cast<size_t>(b) * kD];
-  __shared__ double gs[4][kD];
-  gs[g][c] = t0 + t1;
+  __threadfence();
   __syncthreads();
-  if (g == 0) qbar[hp * kD + c] = static_cast<float>(((gs[0][c] + gs[1][c]) + (gs[2][c] + gs[3][c])) /
-                                                    static_cast<double>(N));
+  if (threadIdx.x == 0) last = atomicAdd(&done[hp], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // four threads per column take every fourth partial, loads batched; fixed order throughout
+  const int c = threadIdx.x & (kD - 1), g = threadIdx.x >> 6;
+  double t = 0.0;
+#pragma unroll 8
+  for (int b2 = g; b2 < static_cast<int>(gridDim.x); b2 += 4) t += __ldcg(&hpart[static_cast<size_t>(b2) * kD + c]);
+  wsum[g][c] = t;
+  __syncthreads();
+  if (g == 0)
+    qbar[hp * kD + c] = static_cast<float>(((wsum[0][c] + wsum[1][c]) + (wsum[2][c] + wsum[3][c])) /
+                                           static_cast<double>(N));
 }
 
 // score_j = qbar . k_j / 8 (fp64 dot, fp32 result); special keys get -inf so they are never ranked.
 // Each block takes a contiguous range of key rows.  Eight lanes per key row, each with one 16-byte
 // chunk (a warp reads 4 whole rows, 512 contiguous bytes, per load), kProbeRowsInFlight rows per
-// lane group loaded before any is used; the 8 partial dots of a row meet in 3 shuffles.  All lanes
+// lane group and step, the next step's requested before this step's are used; the 8 partial dots
+// of a row meet in 3 shuffles.  All lanes
 // of a warp take the same iterations (row validity is a per-group guard), so every shuffle has
 // its whole warp.
 __global__ void __launch_bounds__(256) probe_score_kernel(const uint16_t* __restrict__ k, int N, int V, int ns,
@@ -151,17 +173,24 @@ __global__ void __launch_bounds__(256) probe_score_kernel(const uint16_t* __rest
   const int sub = threadIdx.x & 7, grp = threadIdx.x >> 3;  // 32 row groups per block
   double qv[8];  // this lane's 8 features of qbar, scaled by 2^896 against the 2^-896 of the keys
 #pragma unroll
-  for (int i = 0; i < 8; ++i) qv[i] = static_cast<double>(qbar[hp * kD + 8 * sub + i]) * kBf16Unscale;
+  for (int i = 0; i < 8; ++i) qv[i] = static_cast<double>(qbar[hp * kD + 8 * sub + i]) * kUnscale896;
   const uint4* kh = reinterpret_cast<const uint4*>(k + static_cast<size_t>(h) * N * kD);
   float* sc = scores + static_cast<size_t>(hp) * N;
   const int rows_per = (N + gridDim.x - 1) / gridDim.x;
   const int r0 = blockIdx.x * rows_per, r1 = min(N, r0 + rows_per);
-  for (int jb = r0; jb < r1; jb += 32 * kProbeRowsInFlight) {
-    uint4 w[kProbeRowsInFlight];
+  constexpr int kStep = 32 * kProbeRowsInFlight;
+  uint4 w[kProbeRowsInFlight];
+#pragma unroll
+  for (int f = 0; f < kProbeRowsInFlight; ++f) {
+    const int jf = r0 + 32 * f + grp;  // uniform over the 8 lanes of a row group
+    w[f] = jf < r1 ? kh[static_cast<size_t>(jf) * 8 + sub] : make_uint4(0u, 0u, 0u, 0u);
+  }
+  for (int jb = r0; jb < r1; jb += kStep) {
+    uint4 nx[kProbeRowsInFlight];  // the next step's rows, requested before this step's are used
 #pragma unroll
     for (int f = 0; f < kProbeRowsInFlight; ++f) {
-      const int jf = jb + 32 * f + grp;  // uniform over the 8 lanes of a row group
-      w[f] = jf < r1 ? kh[static_cast<size_t>(jf) * 8 + sub] : make_uint4(0u, 0u, 0u, 0u);
+      const int jf = jb + kStep + 32 * f + grp;
+      nx[f] = jf < r1 ? kh[static_cast<size_t>(jf) * 8 + sub] : make_uint4(0u, 0u, 0u, 0u);
     }
     double d[kProbeRowsInFlight];
 #pragma unroll
@@ -183,6 +212,8 @@ __global__ void __launch_bounds__(256) probe_score_kernel(const uint16_t* __rest
         if (jf < r1) sc[jf] = (jf % V) < ns ? -INFINITY : static_cast<float>(d[f] * 0.125);
       }
     }
+#pragma unroll
+    for (int f = 0; f < kProbeRowsInFlight; ++f) w[f] = nx[f];
   }
 }
 
@@ -480,6 +511,47 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
+// From a 256-bin histogram wh of one digit: the bin holding the remaining-th largest key (bins
+// counted from the top), with `remaining` reduced by the keys of the bins above it.  Lane l sums
+// bins 255 - 8l .. 248 - 8l, a warp scan finds the lane whose bins cross, and that lane walks its
+// eight.  Without a crossing (fewer keys than remaining) the answer is bin 0.
+__device__ __forceinline__ int warp_pick_bin(const int* wh, int lane, int& remaining) {
+  int c[8], local = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = wh[255 - 8 * lane - i];
+    local += c[i];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int above = incl - local;
+  const uint32_t hit = __ballot_sync(0xffffffffu, above < remaining && incl >= remaining);
+  int bin = 0, sub = 0;
+  if (hit == 0) {
+    sub = __shfl_sync(0xffffffffu, incl, 31) - wh[0];
+  } else {
+    const int src = __ffs(hit) - 1;
+    if (lane == src) {
+      int a = above;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        bin = 255 - 8 * lane - i;
+        if (a + c[i] >= remaining) break;
+        a += c[i];
+      }
+      sub = a;
+    }
+    bin = __shfl_sync(0xffffffffu, bin, src);
+    sub = __shfl_sync(0xffffffffu, sub, src);
+  }
+  remaining -= sub;
+  return bin;
+}
+
 // The warp's 8-bit-digit radix select over row[0..T): the key of the kmax-th largest value
 // and how many keys equal to it are taken.  Histogram counts are aggregated per warp
 // instruction (lanes that share a bin add once), so a narrow range of cosines, whose keys
@@ -508,16 +580,17 @@ __device__ __forceinline__ void warp_radix_kth(const float* row, int T, int kmax
       }
     }
     __syncwarp();
-    int b = 255, above = 0;
-    for (; b > 0; --b) {
-      if (above + wh[b] >= remaining) break;
-      above += wh[b];
-    }
-    prefix |= static_cast<uint32_t>(b) << shift;
-    remaining -= above;
+    prefix |= static_cast<uint32_t>(warp_pick_bin(wh, lane, remaining)) << shift;
     mask |= 0xFFu << shift;
     __syncwarp();
   }
+}
+
+// Order-preserving 16-bit key of an fp16 value (larger value -> larger key) and its inverse.
+__device__ __forceinline__ uint32_t order_key16(uint32_t h) { return (h & 0x8000u) ? (~h & 0xFFFFu) : (h | 0x8000u); }
+__device__ __forceinline__ float key16_value(uint32_t key) {
+  const uint32_t h = (key & 0x8000u) ? (key & 0x7FFFu) : (~key & 0xFFFFu);
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
 }
 
 // The kmax largest values of row[0..T) (ties to the lower index) written to out[0..kmax) in
@@ -645,19 +718,24 @@ __global__ void __launch_bounds__(256) unit_features_kernel(const float* __restr
 constexpr float kTokScoreErr = 2e-3f;  // |tensor-core fp16 score - exact cosine| (bound in token_sim.cu)
 constexpr int kTokCap = 64;            // candidates of one (query, frame) the short ranking takes
 
-// This lane's slice of unit vector `row` (features 128c + 4 lane .. +3).
+// This lane's slice of unit vector `row` (features 128c + 4 lane .. +3, as q[4c] .. q[4c + 3]) in
+// fp64, pre-multiplied by 2^896 for products with f32_scaled candidates; 0 past dim.
 __device__ __forceinline__ void load_one_slice(const float* __restrict__ vec, int row, int dim, int lane,
-                                               float4 (&q)[kTkChunks]) {
+                                               double (&q)[4 * kTkChunks]) {
 #pragma unroll
   for (int c = 0; c < kTkChunks; ++c) {
     const int d = 128 * c + 4 * lane;
-    q[c] = d < dim ? ld_f4(vec + static_cast<size_t>(row) * dim + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 f = d < dim ? ld_f4(vec + static_cast<size_t>(row) * dim + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+    q[4 * c] = static_cast<double>(f.x) * kUnscale896;
+    q[4 * c + 1] = static_cast<double>(f.y) * kUnscale896;
+    q[4 * c + 2] = static_cast<double>(f.z) * kUnscale896;
+    q[4 * c + 3] = static_cast<double>(f.w) * kUnscale896;
   }
 }
 
 // fp64 dot of the lane slices q with candidate row fv, summed over the warp (every lane gets
 // the same value: a butterfly adds the same two operands on both sides of each exchange).
-__device__ __forceinline__ double exact_dot(const float4 (&q)[kTkChunks], const float* __restrict__ fv, int dim,
+__device__ __forceinline__ double exact_dot(const double (&q)[4 * kTkChunks], const float* __restrict__ fv, int dim,
                                            int lane) {
   double acc = 0.0;
 #pragma unroll
@@ -665,10 +743,10 @@ __device__ __forceinline__ double exact_dot(const float4 (&q)[kTkChunks], const 
     const int d = 128 * c + 4 * lane;
     if (d < dim) {
       const float4 b = ld_f4(fv + d);
-      acc = fma(static_cast<double>(q[c].x), static_cast<double>(b.x), acc);
-      acc = fma(static_cast<double>(q[c].y), static_cast<double>(b.y), acc);
-      acc = fma(static_cast<double>(q[c].z), static_cast<double>(b.z), acc);
-      acc = fma(static_cast<double>(q[c].w), static_cast<double>(b.w), acc);
+      acc = fma(q[4 * c], f32_scaled(b.x), acc);
+      acc = fma(q[4 * c + 1], f32_scaled(b.y), acc);
+      acc = fma(q[4 * c + 2], f32_scaled(b.z), acc);
+      acc = fma(q[4 * c + 3], f32_scaled(b.w), acc);
     }
   }
 #pragma unroll
@@ -688,7 +766,7 @@ struct TokWarpSmem {
 
 // General ranking of one (query, frame): every candidate within 2 * kTokScoreErr of the
 // approximate kmax-th score gets its exact value, then the whole frame is ranked.
-__device__ void token_rank_general(const __half* __restrict__ seg, int P, int kmax, const float4 (&q)[kTkChunks],
+__device__ void token_rank_general(const __half* __restrict__ seg, int P, int kmax, const double (&q)[4 * kTkChunks],
                                    const float* __restrict__ cand, int dim, const TokWarpSmem& w, int lane,
                                    int32_t* __restrict__ out) {
   for (int v = lane; v < P; v += 32) w.row[v] = __half2float(seg[v]);
@@ -712,7 +790,7 @@ __device__ void token_rank_general(const __half* __restrict__ seg, int P, int km
 }
 
 // Two fp64 dots at once (both rows' loads in flight together); see exact_dot.
-__device__ __forceinline__ void exact_dot2(const float4 (&q)[kTkChunks], const float* __restrict__ f1,
+__device__ __forceinline__ void exact_dot2(const double (&q)[4 * kTkChunks], const float* __restrict__ f1,
                                            const float* __restrict__ f2, int dim, int lane, double& e1, double& e2) {
   float4 b1[kTkChunks], b2[kTkChunks];
 #pragma unroll
@@ -724,15 +802,15 @@ __device__ __forceinline__ void exact_dot2(const float4 (&q)[kTkChunks], const f
   double a1 = 0.0, a2 = 0.0;
 #pragma unroll
   for (int c = 0; c < kTkChunks; ++c) {
-    const double qx = q[c].x, qy = q[c].y, qz = q[c].z, qw = q[c].w;
-    a1 = fma(qx, static_cast<double>(b1[c].x), a1);
-    a2 = fma(qx, static_cast<double>(b2[c].x), a2);
-    a1 = fma(qy, static_cast<double>(b1[c].y), a1);
-    a2 = fma(qy, static_cast<double>(b2[c].y), a2);
-    a1 = fma(qz, static_cast<double>(b1[c].z), a1);
-    a2 = fma(qz, static_cast<double>(b2[c].z), a2);
-    a1 = fma(qw, static_cast<double>(b1[c].w), a1);
-    a2 = fma(qw, static_cast<double>(b2[c].w), a2);
+    const double qx = q[4 * c], qy = q[4 * c + 1], qz = q[4 * c + 2], qw = q[4 * c + 3];
+    a1 = fma(qx, f32_scaled(b1[c].x), a1);
+    a2 = fma(qx, f32_scaled(b2[c].x), a2);
+    a1 = fma(qy, f32_scaled(b1[c].y), a1);
+    a2 = fma(qy, f32_scaled(b2[c].y), a2);
+    a1 = fma(qz, f32_scaled(b1[c].z), a1);
+    a2 = fma(qz, f32_scaled(b2[c].z), a2);
+    a1 = fma(qw, f32_scaled(b1[c].w), a1);
+    a2 = fma(qw, f32_scaled(b2[c].w), a2);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -779,7 +857,7 @@ __device__ __forceinline__ uint32_t chunk_scores(const uint4 w, int c, int e0, i
 // which is the frame's exact ranking.  Otherwise (kmax > 32, or more than kTokCap keys in D)
 // the general ranking runs.
 __device__ void token_rank_frame(const __half* __restrict__ srow, int e0, int P, int kmax,
-                                 const float4 (&q)[kTkChunks], const float* __restrict__ cand, int dim,
+                                 const double (&q)[4 * kTkChunks], const float* __restrict__ cand, int dim,
                                  const TokWarpSmem& w, int lane, int32_t* __restrict__ out) {
   const float band = 2.f * kTokScoreErr;
   const uint4* row4 = reinterpret_cast<const uint4*>(srow);
@@ -946,7 +1024,7 @@ __global__ void __launch_bounds__(256, 3) token_rank_kernel(const __half* __rest
   const int row = blockIdx.x * 8 + warp;
   if (row >= rows) return;
   const int a = r0 + row;
-  float4 q[kTkChunks];
+  double q[4 * kTkChunks];
   load_one_slice(unit, a, dim, lane, q);
   const __half* srow = scores + static_cast<size_t>(row) * ld;
   for (int s = 0; s < S; ++s)
@@ -986,7 +1064,7 @@ __host__ __device__ inline size_t tile_rank_warp_bytes(int T, int kmax) {
 // fp64 dots of the lane slices q with candidate rows idx[0..kN) (idx[j] for j >= n repeats
 // idx[0]), all kN rows' loads in flight together, each summed over the warp.
 template <int kN>
-__device__ __forceinline__ void exact_dots(const float4 (&q)[kTkChunks], const float* __restrict__ cand,
+__device__ __forceinline__ void exact_dots(const double (&q)[4 * kTkChunks], const float* __restrict__ cand,
                                            const int* idx, int n, int dim, int lane, double (&e)[kN]) {
   float4 b[kN][kTkChunks];
 #pragma unroll
@@ -1002,13 +1080,13 @@ __device__ __forceinline__ void exact_dots(const float4 (&q)[kTkChunks], const f
   for (int j = 0; j < kN; ++j) e[j] = 0.0;
 #pragma unroll
   for (int c = 0; c < kTkChunks; ++c) {
-    const double qx = q[c].x, qy = q[c].y, qz = q[c].z, qw = q[c].w;
+    const double qx = q[4 * c], qy = q[4 * c + 1], qz = q[4 * c + 2], qw = q[4 * c + 3];
 #pragma unroll
     for (int j = 0; j < kN; ++j) {
-      e[j] = fma(qx, static_cast<double>(b[j][c].x), e[j]);
-      e[j] = fma(qy, static_cast<double>(b[j][c].y), e[j]);
-      e[j] = fma(qz, static_cast<double>(b[j][c].z), e[j]);
-      e[j] = fma(qw, static_cast<double>(b[j][c].w), e[j]);
+      e[j] = fma(qx, f32_scaled(b[j][c].x), e[j]);
+      e[j] = fma(qy, f32_scaled(b[j][c].y), e[j]);
+      e[j] = fma(qz, f32_scaled(b[j][c].z), e[j]);
+      e[j] = fma(qw, f32_scaled(b[j][c].w), e[j]);
     }
   }
 #pragma unroll
@@ -1034,19 +1112,36 @@ __global__ void __launch_bounds__(256) tile_rank_kernel(const __half* __restrict
   int* widx = hist + 256;                              // [kmax]
   uint32_t* wkey = reinterpret_cast<uint32_t*>(widx + kmax);  // [kmax]
   const int u = r0 + lr;
-  float4 q[kTkChunks];
+  double q[4 * kTkChunks];
   load_one_slice(tilevec, u, dim, lane, q);
+  // the row's approximate cosines as 16-bit order keys (the row buffer's first half), read in
+  // 16-byte chunks (the row starts 16-byte aligned: ld is a multiple of 8)
   const __half* srow = scores + static_cast<size_t>(lr) * ld;
-  for (int v = lane; v < T; v += 32) row[v] = __half2float(srow[v]);
+  uint16_t* keys = reinterpret_cast<uint16_t*>(row);
+  for (int c = lane; 8 * c < T; c += 32) {
+    const uint4 w = *reinterpret_cast<const uint4*>(srow + 8 * c);
+    const uint32_t h[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (8 * c + i < T) keys[8 * c + i] = static_cast<uint16_t>(order_key16((h[i >> 1] >> (16 * (i & 1))) & 0xFFFFu));
+  }
   __syncwarp();
-  uint32_t prefix;
-  int remaining;
-  warp_radix_kth(row, T, kmax, hist, lane, prefix, remaining);
-  const float thr = key_value(prefix) - 2.f * kTokScoreErr;
+  // the kmax-th largest key by bisection: the largest x with at least kmax keys >= x
+  uint32_t lo = 0u, hi = 0xFFFFu;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi + 1u) >> 1;
+    int c = 0;
+    for (int v = lane; v < T; v += 32) c += keys[v] >= mid;
+    if (static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c))) >= kmax) lo = mid;
+    else hi = mid - 1u;
+  }
+  const float thr = key16_value(lo) - 2.f * kTokScoreErr;
+  // candidates: approximate cosine >= thr, i.e. key >= the key of the least fp16 value >= thr
+  const uint32_t thr_key = order_key16(__half_as_ushort(__float2half_ru(thr)));
   int m = 0;
   for (int v0 = 0; v0 < T; v0 += 32) {
     const int v = v0 + lane;
-    const bool take = v < T && row[v] >= thr;
+    const bool take = v < T && keys[v] >= thr_key;
     const uint32_t mask = __ballot_sync(0xffffffffu, take);
     const int pos = m + __popc(mask & ((1u << lane) - 1u));
     if (take && pos < kTrCap) cl[pos] = v;
@@ -1065,9 +1160,22 @@ __global__ void __launch_bounds__(256) tile_rank_kernel(const __half* __restrict
       }
     }
     __syncwarp();
-    warp_rank_row(ev, m, kmax, hist, widx, wkey, lane, out, cl);
+    // rank of each candidate: how many beat it (exact value descending, then tile index
+    // ascending: the list is in index order, so a lower position wins a tie)
+    for (int j = lane; j < m; j += 32) {
+      const uint32_t kj = order_key(ev[j]);
+      int rank = 0;
+      for (int i = 0; i < m; ++i) {
+        const uint32_t ki = order_key(ev[i]);
+        rank += (ki > kj) || (ki == kj && i < j);
+      }
+      if (rank < kmax) out[rank] = cl[j];
+    }
   } else {
-    // every other tile keeps its approximate value, below all exact Top-kmax values
+    // the whole row as fp32 (over the keys, no longer needed); every other tile keeps its
+    // approximate value, below all exact Top-kmax values
+    for (int v = lane; v < T; v += 32) row[v] = __half2float(srow[v]);
+    __syncwarp();
     for (int v0 = 0; v0 < T; v0 += 32) {
       const int v = v0 + lane;
       uint32_t todo = __ballot_sync(0xffffffffu, v < T && row[v] >= thr);
@@ -1083,38 +1191,33 @@ __global__ void __launch_bounds__(256) tile_rank_kernel(const __half* __restrict
   }
 }
 
-__global__ void __launch_bounds__(1024) corr_sort_kernel(const int32_t* __restrict__ ranked, int T, int kmax,
-                                                         int r, int32_t* __restrict__ order) {
-  extern __shared__ unsigned long long keys[];  // [pow2 >= T]
-  int n2 = 1;
-  while (n2 < T) n2 <<= 1;
-  for (int u = threadIdx.x; u < n2; u += blockDim.x) {
-    unsigned long long k = ~0ull;
-    if (u < T) {
-      int mn = 0x7fffffff;
-      for (int i = 0; i < r; ++i) mn = min(mn, ranked[static_cast<size_t>(u) * kmax + i]);
-      k = (static_cast<unsigned long long>(static_cast<uint32_t>(mn)) << 32) | static_cast<uint32_t>(u);
-    }
-    keys[u] = k;
-  }
+// Canonical order of the query tiles for the grouping: by the lowest tile index among the r best
+// of each tile's ranked list, then by tile index.  corr_key_kernel forms each tile's 64-bit key
+// (that minimum over the tile index); corr_rank_kernel gives each tile its position, the number of
+// keys below its own (keys are distinct), with every key of the block held in shared memory.
+__global__ void __launch_bounds__(256) corr_key_kernel(const int32_t* __restrict__ ranked, int T, int kmax, int r,
+                                                       unsigned long long* __restrict__ keys) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= T) return;
+  const int32_t* rr = ranked + static_cast<size_t>(u) * kmax;
+  int mn = 0x7fffffff;
+#pragma unroll 8
+  for (int i = 0; i < r; ++i) mn = min(mn, __ldg(rr + i));
+  keys[u] = (static_cast<unsigned long long>(static_cast<uint32_t>(mn)) << 32) | static_cast<uint32_t>(u);
+}
+
+__global__ void __launch_bounds__(64) corr_rank_kernel(const unsigned long long* __restrict__ keys, int T,
+                                                       int32_t* __restrict__ sorted) {
+  extern __shared__ unsigned long long skeys[];  // [T]
+  for (int v = threadIdx.x; v < T; v += blockDim.x) skeys[v] = keys[v];
   __syncthreads();
-  for (int size = 2; size <= n2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool up = (i & size) == 0;
-          const unsigned long long a = keys[i], b = keys[j];
-          if ((a > b) == up) {
-            keys[i] = b;
-            keys[j] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  for (int u = threadIdx.x; u < T; u += blockDim.x) order[u] = static_cast<int32_t>(keys[u] & 0xffffffffu);
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= T) return;
+  const unsigned long long ku = skeys[u];
+  int rank = 0;
+#pragma unroll 4
+  for (int v = 0; v < T; ++v) rank += skeys[v] < ku;
+  sorted[rank] = u;
 }
 
 __global__ void corr_bitset_kernel(const int32_t* __restrict__ ranked, int T, int kmax, int words,
@@ -1127,32 +1230,44 @@ __global__ void corr_bitset_kernel(const int32_t* __restrict__ ranked, int T, in
   }
 }
 
+// One window of kGroupWindow sorted query tiles: the window's bitsets staged in shared memory
+// (rows of words | 1 words, an odd stride, so the lanes of a warp hit distinct banks), the
+// pairwise intersection counts, then one warp forms greedy groups of four.
 __global__ void __launch_bounds__(256) corr_group_kernel(const uint32_t* __restrict__ bits, int T, int words,
                                                          const int32_t* __restrict__ sorted,
                                                          int32_t* __restrict__ order) {
+  extern __shared__ uint32_t gbits[];  // [kGroupWindow][words | 1]
   __shared__ uint16_t inter[kGroupWindow][kGroupWindow];
   __shared__ int tiles[kGroupWindow];
+  const int ws = words | 1;
   const int w0 = blockIdx.x * kGroupWindow;
   const int n = min(kGroupWindow, T - w0);
   for (int i = threadIdx.x; i < n; i += blockDim.x) tiles[i] = sorted[w0 + i];
   __syncthreads();
+  for (int e = threadIdx.x; e < n * words; e += blockDim.x) {
+    const int a = e / words, w = e - a * words;
+    gbits[a * ws + w] = bits[static_cast<size_t>(tiles[a]) * words + w];
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
     const int a = e / n, b = e - a * n;
     if (b < a) continue;
-    const uint32_t* ba = bits + static_cast<size_t>(tiles[a]) * words;
-    const uint32_t* bb = bits + static_cast<size_t>(tiles[b]) * words;
+    const uint32_t* ba = gbits + a * ws;
+    const uint32_t* bb = gbits + b * ws;
     int c = 0;
     for (int w = 0; w < words; ++w) c += __popc(ba[w] & bb[w]);
     inter[a][b] = inter[b][a] = static_cast<uint16_t>(min(c, 65535));
   }
   __syncthreads();
   if (threadIdx.x >= 32) return;
-  // one warp: greedy groups of four inside the window; lane l owns candidates l and l + 32
+  // one warp: greedy groups of four inside the window; lane l owns candidates l and l + 32.  A
+  // candidate's key packs its score over the position from the end, so the warp maximum is the
+  // highest score, ties to the earlier position; 0 marks a candidate already taken.
   const int lane = threadIdx.x;
   bool left0 = lane < n, left1 = lane + 32 < n;
   int out = w0;
   for (int u = 0; u < n; ++u) {
-    const bool u_left = __shfl_sync(0xffffffffu, (u & 31) < 32 ? ((u < 32) ? left0 : left1) : false, u & 31);
+    const bool u_left = __shfl_sync(0xffffffffu, u < 32 ? left0 : left1, u & 31);
     if (!u_left) continue;
     if (lane == (u & 31)) {
       if (u < 32) left0 = false; else left1 = false;
@@ -1162,20 +1277,11 @@ __global__ void __launch_bounds__(256) corr_group_kernel(const uint32_t* __restr
     int sc0 = left0 ? inter[u][lane] : -1;
     int sc1 = left1 ? inter[u][lane + 32] : -1;
     for (int k = 0; k < 3; ++k) {
-      // argmax over the window (ties to the earlier position)
-      int best = sc0 >= sc1 ? sc0 : sc1;
-      int pos = sc0 >= sc1 ? lane : lane + 32;
-      if (best < 0) pos = 1 << 20;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const int ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int op = __shfl_xor_sync(0xffffffffu, pos, o);
-        if (ob > best || (ob == best && op < pos)) {
-          best = ob;
-          pos = op;
-        }
-      }
-      if (best < 0) break;
+      const uint32_t k0 = sc0 >= 0 ? (static_cast<uint32_t>(sc0) << 7) | static_cast<uint32_t>(127 - lane) : 0u;
+      const uint32_t k1 = sc1 >= 0 ? (static_cast<uint32_t>(sc1) << 7) | static_cast<uint32_t>(95 - lane) : 0u;
+      const uint32_t best = __reduce_max_sync(0xffffffffu, max(k0, k1));
+      if (best == 0u) break;
+      const int pos = 127 - static_cast<int>(best & 127u);
       if (lane == 0) order[out] = tiles[pos];
       ++out;
       if (pos == lane) left0 = false;
@@ -1224,7 +1330,7 @@ TokWs token_ws(long long R, int dim) {
 }
 
 // Correspondence part of the select workspace, offsets from its (256-byte aligned) start: fp32 tile
-// unit vectors [T][dim], grouping bitsets [T][words], sorted tiles [T]; with the tensor-core
+// unit vectors [T][dim], grouping bitsets [T][words], sorted tiles [T], their sort keys [T]; with the tensor-core
 // cosines (dim <= 384) also fp16 tile unit vectors [T][dim16] (zero-padded to a multiple of 64
 // features) and the fp16 cosines of one chunk of query tiles [chunk_rows][ld] (ld = T rounded up
 // to 8; chunks of at most kTileScoreBudget bytes).
@@ -1234,7 +1340,7 @@ struct CorrWs {
   bool tc;
   int dim16, chunk_rows;
   long long ld;
-  size_t tilevec, bits, sorted, tile16, scores, end;
+  size_t tilevec, bits, sorted, keys, tile16, scores, end;
 };
 
 CorrWs corr_ws(int T, int dim) {
@@ -1249,7 +1355,8 @@ CorrWs corr_ws(int T, int dim) {
   c.tilevec = 0;
   c.bits = al(static_cast<size_t>(T) * dim * sizeof(float));
   c.sorted = al(c.bits + static_cast<size_t>(T) * ((T + 31) / 32) * sizeof(uint32_t));
-  c.end = al(c.sorted + static_cast<size_t>(T) * sizeof(int32_t));
+  c.keys = al(c.sorted + static_cast<size_t>(T) * sizeof(int32_t));
+  c.end = al(c.keys + static_cast<size_t>(T) * sizeof(unsigned long long));
   c.tile16 = c.scores = c.end;
   if (c.tc) {
     c.scores = al(c.tile16 + static_cast<size_t>(T) * c.dim16 * 2);
@@ -1258,9 +1365,10 @@ CorrWs corr_ws(int T, int dim) {
   return c;
 }
 
-// Probe Top-K scratch: digit histograms and pass counters (zeroed per build), per-chunk counts.
+// Probe scratch: digit histograms and pass counters (zeroed per build, with one more counter per
+// head for the mean's partial sums), per-chunk counts.
 size_t rank_zero_bytes(int n_probe) {
-  return static_cast<size_t>(n_probe) * kRankPasses * (kRankBins * sizeof(int) + sizeof(unsigned));
+  return static_cast<size_t>(n_probe) * (kRankPasses * (kRankBins * sizeof(int) + sizeof(unsigned)) + sizeof(unsigned));
 }
 size_t rank_counts_bytes(int n_probe, int N) {
   return static_cast<size_t>(n_probe) * ((N + kRankChunk - 1) / kRankChunk) * 2 * sizeof(int);
@@ -1316,6 +1424,7 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
   off = (off + 255) & ~size_t(255);
   int* rank_hist = reinterpret_cast<int*>(ws + off);  // zeroed with rank_done in one memset
   unsigned* rank_done = reinterpret_cast<unsigned*>(rank_hist + static_cast<size_t>(sp.n_probe) * kRankPasses * kRankBins);
+  unsigned* mean_done = rank_done + static_cast<size_t>(sp.n_probe) * kRankPasses;
   off += rank_zero_bytes(sp.n_probe);
   off = (off + 255) & ~size_t(255);
   RankState* rank_state = reinterpret_cast<RankState*>(ws + off);
@@ -1334,21 +1443,27 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
       a.k[i] = sp.probe_k[i];
       a.cache_off[i] = sp.probe_off[i];
     }
-    probe_partial_kernel<<<dim3(kProbePartials, sp.n_probe), 256, 0, stream>>>(q, sp.N, a, partial);
-    probe_mean_kernel<<<sp.n_probe, 4 * kD, 0, stream>>>(partial, kProbePartials, sp.N, qbar);
-    // contiguous ranges of key rows, 32 x kProbeRowsInFlight rows per block and step
-    const int score_blocks = std::max(1, std::min((sp.N + 127) / 128, 2 * sp.num_sms));
-    probe_score_kernel<<<dim3(score_blocks, sp.n_probe), 256, 0, stream>>>(k, sp.N, sp.V, sp.ns, a, qbar, scores);
-    const int rank_blocks = (sp.N + kRankChunk - 1) / kRankChunk;
     cudaError_t e = cudaMemsetAsync(rank_hist, 0, rank_zero_bytes(sp.n_probe), stream);
     if (e != cudaSuccess) return e;
+    // one wave: as many blocks per head as the SMs hold at once, split over the probe heads
+    int occ_mean = 1, occ_score = 1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_mean, probe_mean_kernel, 256, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_score, probe_score_kernel, 256, 0);
+    const int mean_blocks =
+        std::max(1, std::min(kProbePartials, std::max(1, occ_mean) * sp.num_sms / sp.n_probe));
+    probe_mean_kernel<<<dim3(mean_blocks, sp.n_probe), 256, 0, stream>>>(q, sp.N, a, partial, mean_done, qbar);
+    // contiguous ranges of key rows, 32 x kProbeRowsInFlight rows per block and step
+    const int score_blocks =
+        std::max(1, std::min((sp.N + 127) / 128, std::max(1, occ_score) * sp.num_sms / sp.n_probe));
+    probe_score_kernel<<<dim3(score_blocks, sp.n_probe), 256, 0, stream>>>(k, sp.N, sp.V, sp.ns, a, qbar, scores);
+    const int rank_blocks = (sp.N + kRankChunk - 1) / kRankChunk;
     for (int pass = 0; pass < kRankPasses; ++pass)
       probe_digit_kernel<<<dim3(rank_blocks, sp.n_probe), 256, 0, stream>>>(scores, sp.N, a, pass, rank_hist,
                                                                            rank_done, rank_state);
     probe_count_kernel<<<dim3(rank_blocks, sp.n_probe), 256, 0, stream>>>(scores, sp.N, rank_state, rank_counts);
     probe_write_kernel<<<dim3(rank_blocks, sp.n_probe), 256, 0, stream>>>(scores, sp.N, a, rank_state, rank_counts,
                                                                          cache);
-    *n_launch += 3 + kRankPasses + 2;
+    *n_launch += 2 + kRankPasses + 2;
   }
   if (sp.corr_kmax > 0) {
     const CorrWs cw = corr_ws(sp.T, sp.dim);
@@ -1410,19 +1525,22 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
     int32_t* sorted = reinterpret_cast<int32_t*>(cbase + cw.sorted);
     int32_t* order = cache + sp.order_off;
     if (sp.T <= kMaxSortTiles) {
-      int n2 = 1;
-      while (n2 < sp.T) n2 <<= 1;
-      const size_t ssmem = sizeof(unsigned long long) * n2;
-      e = cudaFuncSetAttribute(corr_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssmem));
+      unsigned long long* gkeys = reinterpret_cast<unsigned long long*>(cbase + cw.keys);
+      corr_key_kernel<<<(sp.T + 255) / 256, 256, 0, stream>>>(cache + sp.corr_off, sp.T, sp.corr_kmax,
+                                                               sp.corr_kmax > 1 ? sp.corr_kmax / 2 : 1, gkeys);
+      const size_t ksmem = sizeof(unsigned long long) * static_cast<size_t>(sp.T);
+      e = cudaFuncSetAttribute(corr_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ksmem));
       if (e != cudaSuccess) return e;
-      corr_sort_kernel<<<1, 1024, ssmem, stream>>>(cache + sp.corr_off, sp.T, sp.corr_kmax,
-                                                   sp.corr_kmax > 1 ? sp.corr_kmax / 2 : 1, sorted);
+      corr_rank_kernel<<<(sp.T + 63) / 64, 64, ksmem, stream>>>(gkeys, sp.T, sorted);
       e = cudaMemsetAsync(bits, 0, static_cast<size_t>(sp.T) * words * sizeof(uint32_t), stream);
       if (e != cudaSuccess) return e;
       corr_bitset_kernel<<<148, 256, 0, stream>>>(cache + sp.corr_off, sp.T, sp.corr_kmax, words, bits);
-      corr_group_kernel<<<(sp.T + kGroupWindow - 1) / kGroupWindow, 256, 0, stream>>>(bits, sp.T, words, sorted,
-                                                                                      order);
-      *n_launch += 3;
+      const size_t gsmem = sizeof(uint32_t) * kGroupWindow * static_cast<size_t>(words | 1);
+      e = cudaFuncSetAttribute(corr_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(gsmem));
+      if (e != cudaSuccess) return e;
+      corr_group_kernel<<<(sp.T + kGroupWindow - 1) / kGroupWindow, 256, gsmem, stream>>>(bits, sp.T, words, sorted,
+                                                                                          order);
+      *n_launch += 4;
     } else {
       identity_order_kernel<<<(sp.T + 255) / 256, 256, 0, stream>>>(sp.T, order);
       *n_launch += 1;

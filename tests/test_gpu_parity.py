@@ -221,6 +221,38 @@ def test_probe_ties_go_to_the_lower_index(n_rows):
     check_rows(case, heads, sels, out, lambda h: np.arange(L.N))
 
 
+@pytest.mark.parametrize("n_rows", [2, 3])
+def test_probe_ties_span_key_chunks(n_rows):
+    """As above on a layer of 12,840 keys, so a tie group is spread over every 4,096-key chunk
+    of the multi-block radix select: the equal keys taken must be the lowest-index ones across
+    chunks, not within each chunk.  Budgets cut through a tie group (k = 5000 and 4300 with 2 or
+    3 groups of ~4,300-6,400 keys)."""
+    heads = [HeadCfg(PROBE, k=5000), HeadCfg(PROBE, k=4300), HeadCfg(PROBE, k=1), HeadCfg(SCAN, stride=4, phase=3)]
+    case = Case(_custom(8, 40, heads, seed=90 + n_rows))
+    L = case.L
+    assert L.N > 3 * 4096
+    rng = np.random.default_rng(900 + n_rows)
+    patch = O.patch_tokens(L)
+    tmpl = patch[rng.choice(len(patch), size=n_rows, replace=False)]
+    src = np.arange(L.N)
+    src[patch] = tmpl[rng.integers(0, n_rows, size=len(patch))]
+    src_t = torch.from_numpy(src).cuda()
+    for h in range(3):
+        case.k[h] = case.k[h][src_t]
+    case.K = bf16_to_f32(case.k)
+    att, out = run_gpu(case, heads)
+    sel = oracle_select(case, heads)
+    for h in range(3):
+        sc = sel.probe_scores[h][patch]
+        kth = np.sort(sc)[::-1][heads[h].k - 1]
+        tied = patch[sc == kth]
+        assert len(tied) > 1 and tied.min() < 4096 and tied.max() >= 3 * 4096
+    sels = check_selection(case, heads, att, sel)
+    assert not sels.over_gpu, f"probe heads {sels.over_gpu} broke a tie differently from the oracle"
+    rows = np.sort(rng.choice(L.N, size=384, replace=False))
+    check_rows(case, heads, sels, out, lambda h: rows)
+
+
 @pytest.mark.parametrize("period", [2, 3])
 def test_tile_ties_go_to_the_lower_index(period):
     """Views s and s + period get the same DINO features on a layout whose views are exactly two
