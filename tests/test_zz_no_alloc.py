@@ -13,18 +13,28 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 
+def _workload(name):
+    from saf3r_synth import CORR, PROBE, TOKEN, WORKLOADS, HeadCfg, Layout, Workload
+    if name == "tiny_token":
+        # token-wise heads (two per-frame budgets) beside a probe and a correspondence head
+        return Workload("tiny_token", Layout(S=4, g=16, H=4), M=512, delta=37, D=256,
+                        heads=[HeadCfg(TOKEN, k=8), HeadCfg(PROBE, k=128), HeadCfg(CORR, k=4), HeadCfg(TOKEN, k=4)],
+                        seed=1234)
+    return WORKLOADS[name]
+
+
 def _inputs(name):
-    from saf3r_synth import WORKLOADS, Scene, qkv
-    wl = WORKLOADS[name]
+    from saf3r_synth import Scene, qkv
+    wl = _workload(name)
     scene = Scene(wl)
     q, k, v = qkv(scene, 0, device="cuda")
     return wl, q, k, v, torch.from_numpy(scene.dino()).cuda()
 
 
-@pytest.mark.parametrize("name", ["tiny", "s32"])
+@pytest.mark.parametrize("name", ["tiny", "s32", "tiny_token"])
 def test_static_select_matches_regular_on_two_calls(name):
     import head_wise_dynamic_b200 as hw
-    from saf3r_synth import CORR, PROBE
+    from saf3r_synth import CORR, PROBE, TOKEN
     wl, q, k, v, dino = _inputs(name)
     L = hw.layout_of(wl.layout)
     cfg = hw.cfg_array(wl.heads)
@@ -43,7 +53,7 @@ def test_static_select_matches_regular_on_two_calls(name):
         torch.cuda.synchronize()
         hw.saf3r_check()
         for h, hc in enumerate(wl.heads):
-            if hc.kind in (PROBE, CORR):
+            if hc.kind in (PROBE, CORR, TOKEN):
                 a = hw.saf3r_cache_export(L, cfg, cache, h)
                 b = hw.saf3r_cache_export(L, cfg, ref, h)
                 assert np.array_equal(a, b), f"call {call}: head {h} index list differs"
