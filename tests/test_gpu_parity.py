@@ -277,6 +277,27 @@ def test_tile_ties_go_to_the_lower_index(period):
     check_rows(case, heads, sels, out, lambda h: np.arange(L.N))
 
 
+def test_tile_rank_with_more_candidates_than_its_list():
+    """Every patch gets the same DINO feature on a 160-view layout of two-tile views (T = 320), so
+    every tile mean is the same vector and each query tile's row holds T candidates within the
+    tensor-core bound of its k-th cosine: more than the ranking kernel's list of 256, so the row
+    is recomputed in place (its second path).  The oracle's means are exactly equal (all ties, the
+    lowest tile indices win); the GPU's fp32 means may differ in the last bits, so its lists are
+    accepted within the boundary band and the outputs compared over them."""
+    heads = [HeadCfg(CORR, k=64), HeadCfg(CORR, k=300), HeadCfg(HYBRID, k=7, stride=9, phase=4),
+             HeadCfg(POSITION)]
+    case = Case(_custom(160, 11, heads, seed=85, ns=7))
+    L = case.L
+    assert L.V == 128 and L.T == 320
+    case.dino = case.dino[:1].expand(L.S * L.P, L.dino_dim).contiguous()
+    att, out = run_gpu(case, heads)
+    sel = oracle_select(case, heads)
+    assert np.all(sel.tile_cos == sel.tile_cos[0, 0])  # every cosine ties in the oracle
+    sels = check_selection(case, heads, att, sel)
+    rows = np.sort(np.random.default_rng(850).choice(L.N, size=256, replace=False))
+    check_rows(case, heads, sels, out, lambda h: rows)
+
+
 # ---------------------------------------------------------------- token-wise per-frame DINO Top-K
 
 TOKEN_CASES = {
