@@ -1206,18 +1206,20 @@ __global__ void __launch_bounds__(256) corr_key_kernel(const int32_t* __restrict
   keys[u] = (static_cast<unsigned long long>(static_cast<uint32_t>(mn)) << 32) | static_cast<uint32_t>(u);
 }
 
-__global__ void __launch_bounds__(64) corr_rank_kernel(const unsigned long long* __restrict__ keys, int T,
-                                                       int32_t* __restrict__ sorted) {
+__global__ void __launch_bounds__(256) corr_rank_kernel(const unsigned long long* __restrict__ keys, int T,
+                                                        int32_t* __restrict__ sorted) {
   extern __shared__ unsigned long long skeys[];  // [T]
   for (int v = threadIdx.x; v < T; v += blockDim.x) skeys[v] = keys[v];
   __syncthreads();
-  const int u = blockIdx.x * blockDim.x + threadIdx.x;
-  if (u >= T) return;
-  const unsigned long long ku = skeys[u];
+  // four threads per tile, each counting over every fourth key; a shuffle pair adds the four
+  const int u = blockIdx.x * (blockDim.x >> 2) + (threadIdx.x >> 2), part = threadIdx.x & 3;
+  const unsigned long long ku = u < T ? skeys[u] : 0ull;
   int rank = 0;
 #pragma unroll 4
-  for (int v = 0; v < T; ++v) rank += skeys[v] < ku;
-  sorted[rank] = u;
+  for (int v = part; v < T; v += 4) rank += skeys[v] < ku;
+  rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+  rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+  if (u < T && part == 0) sorted[rank] = u;
 }
 
 __global__ void corr_bitset_kernel(const int32_t* __restrict__ ranked, int T, int kmax, int words,
@@ -1531,7 +1533,7 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
       const size_t ksmem = sizeof(unsigned long long) * static_cast<size_t>(sp.T);
       e = cudaFuncSetAttribute(corr_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ksmem));
       if (e != cudaSuccess) return e;
-      corr_rank_kernel<<<(sp.T + 63) / 64, 64, ksmem, stream>>>(gkeys, sp.T, sorted);
+      corr_rank_kernel<<<(sp.T + 63) / 64, 256, ksmem, stream>>>(gkeys, sp.T, sorted);
       e = cudaMemsetAsync(bits, 0, static_cast<size_t>(sp.T) * words * sizeof(uint32_t), stream);
       if (e != cudaSuccess) return e;
       corr_bitset_kernel<<<148, 256, 0, stream>>>(cache + sp.corr_off, sp.T, sp.corr_kmax, words, bits);
