@@ -43,28 +43,56 @@ __device__ __forceinline__ void load16(const uint16_t* p, float (&x)[16]) {
   }
 }
 
-__device__ __forceinline__ int special_tok(int r, int V, int ns) {
-  const int s = r / ns;
-  return s * V + (r - s * ns);
-}
+// n / d and n % d for a divisor fixed per row: one multiply-high by m = ceil(2^32 / d) (exact for
+// n < 2^32 / d, which holds for every key rank here; one correction step covers the rest), the
+// divisor 1 on its own path.
+struct Divider {
+  uint32_t d, m;
+  __device__ explicit Divider(uint32_t dd) : d(dd), m(dd > 1u ? 0xFFFFFFFFu / dd + 1u : 0u) {}
+  __device__ __forceinline__ uint32_t div(uint32_t n, uint32_t& r) const {
+    if (d == 1u) {
+      r = 0u;
+      return n;
+    }
+    uint32_t q = __umulhi(n, m);
+    int rr = static_cast<int>(n - q * d);
+    if (rr < 0) {
+      --q;
+      rr += static_cast<int>(d);
+    } else if (rr >= static_cast<int>(d)) {
+      ++q;
+      rr -= static_cast<int>(d);
+    }
+    r = static_cast<uint32_t>(rr);
+    return q;
+  }
+};
 
 // Token of kept key n of a patch query: ranks n < nl come from the per-frame lists (frame n / kf),
-// the rest are the special tokens.  An out-of-range list entry is recorded in the error word and
-// read as patch 0 (the group stays converged).
-__device__ __forceinline__ int key_token(const TokenAttnParams& p, const int32_t* lists, int n, int nl, int kf) {
-  if (n >= nl) return special_tok(n - nl, p.V, p.ns);
-  const int s = n / kf, r = n - s * kf;
-  int pp = lists[s * p.tok_kmax + r];
+// the rest are the special tokens (view by view).  An out-of-range list entry is recorded in the
+// error word and read as patch 0 (the group stays converged).
+__device__ __forceinline__ int key_token(const TokenAttnParams& p, const int32_t* lists, int n, int nl,
+                                         const Divider& by_kf, const Divider& by_ns) {
+  uint32_t r;
+  if (n >= nl) {
+    const uint32_t s = by_ns.div(static_cast<uint32_t>(n - nl), r);
+    return static_cast<int>(s) * p.V + static_cast<int>(r);
+  }
+  const uint32_t s = by_kf.div(static_cast<uint32_t>(n), r);
+  int pp = lists[static_cast<int>(s) * p.tok_kmax + static_cast<int>(r)];
   if (pp < 0 || pp >= p.P) {
     atomicCAS(p.err, 0, SAF3R_ERR_INDEX);
     pp = 0;
   }
-  return s * p.V + p.ns + pp;
+  return static_cast<int>(s) * p.V + p.ns + pp;
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(256) token_attn_kernel(const TokenAttnParams p) {
+// Four blocks per SM (64 registers; a few spill): more warps to hide the gathers' L2 latency
+// measured faster than three blocks at 80 registers without spills (S=32 token layer 4.39-4.52 vs
+// 4.58-4.68 ms).
+__global__ void __launch_bounds__(256, 4) token_attn_kernel(const TokenAttnParams p) {
   if (p.ok_flag != nullptr && *p.ok_flag == 0) return;  // cache check failed: leave `out` untouched
   const int lane = threadIdx.x & 31;
   const int grp = lane >> 2, sub = lane & 3;            // key group, feature quarter [16*sub, 16*sub+16)
@@ -79,6 +107,7 @@ __global__ void __launch_bounds__(256) token_attn_kernel(const TokenAttnParams p
     const int a = static_cast<int>(task - static_cast<long long>(hi) * R);  // patch row a = s*P + patch
     const int i = (a / p.P) * p.V + p.ns + (a % p.P);
     const int h = p.heads[hi], kf = p.k[hi];  // kf: per-frame budget of this head
+    const Divider by_kf(static_cast<uint32_t>(kf)), by_ns(static_cast<uint32_t>(p.ns > 0 ? p.ns : 1));
     const size_t hb = static_cast<size_t>(h) * p.N * kD;
     const int nl = p.S * kf;  // ranked keys; the special tokens follow
     const int nk = nl + nsp;
@@ -91,8 +120,8 @@ __global__ void __launch_bounds__(256) token_attn_kernel(const TokenAttnParams p
     for (int c = 0; c < 16; ++c) o[c] = 0.f;
     for (int n = grp; n < nk; n += 16) {
       const bool two = n + 8 < nk;
-      const int tok0 = key_token(p, lists, n, nl, kf);
-      const int tok1 = two ? key_token(p, lists, n + 8, nl, kf) : tok0;
+      const int tok0 = key_token(p, lists, n, nl, by_kf, by_ns);
+      const int tok1 = two ? key_token(p, lists, n + 8, nl, by_kf, by_ns) : tok0;
       float k0[16], k1[16], v0[16], v1[16];
       load16(p.k_ + hb + static_cast<size_t>(tok0) * kD + 16 * sub, k0);
       load16(p.k_ + hb + static_cast<size_t>(tok1) * kD + 16 * sub, k1);
