@@ -438,3 +438,36 @@ def test_given_token_lists_replace_the_ranking():
     diff = set(O.key_set(L, hc, sel, 0, i).tolist()) ^ set(O.key_set(L, hc, given, 0, i).tolist())
     assert diff == {1 * L.V + L.n_special + old, 1 * L.V + L.n_special + new}
     assert np.array_equal(O.key_set(L, hc, sel, 0, i + 1), O.key_set(L, hc, given, 0, i + 1))
+
+
+def test_nmse_sample_estimate_within_its_standard_error():
+    """eq. 1's NMSE on all query rows against its row-sample estimate.  On a layer small enough for
+    every row: (1) the all-row table equals sum_i |O_f,i - O_s,i|^2 / sum_i |O_f,i|^2 with the dense
+    rows from torch's fp64 SDPA; (2) a 300-row sample's value (a ratio estimate) lies within 6
+    standard errors of it, the error estimated from the per-row terms, for every head and
+    candidate.  This pins the sampled form used at full size by its sampling distribution."""
+    L = Layout(S=4, g=20, H=2)
+    rng = np.random.default_rng(99)
+    Q, K, V = (rng.standard_normal((L.H, L.N, 64)) for _ in range(3))
+    dino = rng.standard_normal((L.S * L.P, L.dino_dim)).astype(np.float32)
+    cands = [HeadCfg(PROBE, k=150), HeadCfg(SCAN, stride=4), HeadCfg(POSITION), HeadCfg(CORR, k=3)]
+    every = [np.arange(L.N)] * L.H
+    table = O.nmse_table_sampled(L, cands, Q, K, V, dino, every)
+    n = 300
+    sample = [np.sort(rng.choice(L.N, size=n, replace=False)) for _ in range(L.H)]
+    est = O.nmse_table_sampled(L, cands, Q, K, V, dino, sample)
+    for h in range(L.H):
+        q = torch.from_numpy(Q[h])[None, None]
+        dense = torch.nn.functional.scaled_dot_product_attention(
+            q, torch.from_numpy(K[h])[None, None], torch.from_numpy(V[h])[None, None], scale=0.125)[0, 0].numpy()
+        for c, cand in enumerate(cands):
+            hc = O.apply_candidate(cand, h)
+            heads = [O.apply_candidate(cand, x) for x in range(L.H)]
+            sel = O.select(L, heads, Q, K, dino)
+            sparse = O.sparse_rows(L, hc, sel, h, Q[h], K[h], V[h], np.arange(L.N))
+            a = np.sum((dense - sparse) ** 2, axis=1)
+            b = np.sum(dense ** 2, axis=1)
+            R = a.sum() / b.sum()
+            assert abs(table[h, c] - R) <= 1e-9 * max(R, 1e-12), (h, c, table[h, c], R)
+            se = math.sqrt((1.0 - n / L.N) * np.var(a - R * b) / n) / b.mean()
+            assert abs(est[h, c] - R) <= 6.0 * se + 1e-12, (h, c, est[h, c], R, se)
