@@ -219,6 +219,10 @@ struct SparseLayout {
   long long kc_rows = 0, qc_rows = 0, seg_total = 0, cnt_total = 0;
   int off_total = 0;
   std::vector<int> kc_begin, n_rows, qc_begin, n_lat, n_off, off_list;
+  // token-wise heads whose patch queries' special keys run in the tensor-core kernel (one extra
+  // plan each, while the plans fit), with their partial outputs in the workspace
+  std::vector<int> use_part;
+  std::vector<size_t> part_o_off, part_lse_off;
   // shared plan lists
   struct List {
     int kind, param, tail, cap, n_items;  // tail: rows of the derived run that ends every item (tile lists)
@@ -246,7 +250,19 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
   s.n_off.assign(H, 0);
   s.off_list.assign(H, 0);
   s.list_of.assign(H, -1);
+  s.use_part.assign(H, 0);
+  s.part_o_off.assign(H, 0);
+  s.part_lse_off.assign(H, 0);
   const int nsp = d.ns * d.S;
+  {
+    int plans = 0;  // plans of the tensor-core kernel without the extra ones
+    for (int h = 0; h < H; ++h) plans += cfg[h].type != SAF3R_TOKEN || nsp > 0;
+    for (int h = 0; h < H; ++h)
+      if (cfg[h].type == SAF3R_TOKEN && nsp > 0 && plans < kMaxHeads) {
+        s.use_part[h] = 1;
+        ++plans;
+      }
+  }
   for (int h = 0; h < H; ++h) {
     const saf3r_head_cfg& c = cfg[h];
     int rows = 0;
@@ -259,11 +275,13 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
       case SAF3R_PROBE:
         rows = nsp + c.k;
         break;
-      case SAF3R_TOKEN:  // the special-token queries, gathered for the tensor-core kernel
+      case SAF3R_TOKEN:  // the special-token queries, gathered for the tensor-core kernel, and
+                         // the special keys of the patch queries' partial plan
         if (nsp > 0) {
           s.qc_begin[h] = static_cast<int>(s.qc_rows);
           s.qc_rows += nsp;
         }
+        if (s.use_part[h]) rows = nsp;
         break;
       case SAF3R_SCAN:
       case SAF3R_HYBRID: {  // the lattice, then the specials off it
@@ -328,6 +346,14 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
   off = align256(off + static_cast<size_t>(s.seg_total) * sizeof(Seg));
   s.cnt_off = off;
   off = align256(off + static_cast<size_t>(s.cnt_total) * 4);
+  for (int h = 0; h < H; ++h) {
+    if (!s.use_part[h]) continue;
+    const size_t rows = static_cast<size_t>(d.S) * d.P;
+    s.part_o_off[h] = off;
+    off = align256(off + rows * kD * sizeof(float));
+    s.part_lse_off[h] = off;
+    off = align256(off + rows * sizeof(float));
+  }
   s.total = off;
   return s;
 }
@@ -429,37 +455,51 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   // attention
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
-  // the patch queries of token-wise heads run in their own kernel (no shared key runs); their
-  // special-token queries (every key: dense rows) and every other head in the MMA kernel
-  std::vector<int> order;
+  // the patch queries of token-wise heads run in their own kernel (no shared key runs) over their
+  // per-frame lists; their special keys (a dense block: every patch query keeps them) run here as
+  // a partial plan merged by that kernel, and their special-token queries (every key: dense rows)
+  // and every other head run here as well
+  struct PlanRef {
+    int h;
+    bool part;
+  };
+  std::vector<PlanRef> order;
   TokenAttnParams tp;
   std::memset(&tp, 0, sizeof(tp));
   for (int h = 0; h < d.H; ++h) {
     if (cfg[h].type == SAF3R_TOKEN) {
       tp.heads[tp.n_heads] = h;
       tp.k[tp.n_heads] = cfg[h].k;
+      if (s.use_part[h]) {
+        tp.part_o[tp.n_heads] = reinterpret_cast<const float*>(ws + s.part_o_off[h]);
+        tp.part_lse[tp.n_heads] = reinterpret_cast<const float*>(ws + s.part_lse_off[h]);
+        order.push_back({h, true});
+      }
       ++tp.n_heads;
-      if (s.qc_begin[h] >= 0) order.push_back(h);
+      if (s.qc_begin[h] >= 0) order.push_back({h, false});
     } else {
-      order.push_back(h);
+      order.push_back({h, false});
     }
   }
+  const int nsp = d.ns * d.S;
+  auto plan_keys = [&](const PlanRef& r) { return r.part ? static_cast<double>(nsp) : est_keys(d, cfg[r.h], s, r.h); };
   std::stable_sort(order.begin(), order.end(),
-                   [&](int a, int b) { return est_keys(d, cfg[a], s, a) > est_keys(d, cfg[b], s, b); });
+                   [&](const PlanRef& a, const PlanRef& b) { return plan_keys(a) > plan_keys(b); });
   const int n_main = static_cast<int>(order.size());
   int item = 0;
   for (int i = 0; i < n_main; ++i) {
-    const int h = order[i];
+    const int h = order[i].h;
+    const bool part = order[i].part;
     const saf3r_head_cfg& c = cfg[h];
     HeadPlan& hp = p.heads[i];
     hp.head = h;
     hp.kind = c.type;
-    hp.q_src = c.type == SAF3R_POSITION ? 1 : (tile_kind(c.type) ? 2 : (c.type == SAF3R_TOKEN ? 3 : 0));
-    hp.q_base = tile_kind(c.type) ? cl.order_off : (s.qc_begin[h] < 0 ? 0 : s.qc_begin[h]);
+    hp.q_src = part ? 0 : (c.type == SAF3R_POSITION ? 1 : (tile_kind(c.type) ? 2 : (c.type == SAF3R_TOKEN ? 3 : 0)));
+    hp.q_base = part ? 0 : (tile_kind(c.type) ? cl.order_off : (s.qc_begin[h] < 0 ? 0 : s.qc_begin[h]));
     hp.lat_stride = c.type == SAF3R_HYBRID ? c.stride : 0;
     hp.lat_phase = c.type == SAF3R_HYBRID ? c.phase : 0;
     hp.kc_base = s.kc_begin[h];
-    hp.n_items = c.type == SAF3R_TOKEN ? items_of(d.ns * d.S) : items_of(d.N);
+    hp.n_items = (c.type == SAF3R_TOKEN && !part) ? items_of(d.ns * d.S) : items_of(d.N);
     hp.item_begin = item;
     item += hp.n_items;
     hp.seg_list = -1;
@@ -467,6 +507,16 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     hp.cnt_list = 0;
     hp.radius = c.radius;
     hp.nb_base = d.ns * d.S + d.P;
+    hp.part_o = nullptr;
+    hp.part_lse = nullptr;
+    if (part) {
+      // every query row against the head's derived special rows; the patch rows' results go to
+      // the partial buffers
+      hp.seg = Seg{1, 0, nsp, kSegAllQuarters};
+      hp.part_o = reinterpret_cast<float*>(ws + s.part_o_off[h]);
+      hp.part_lse = reinterpret_cast<float*>(ws + s.part_lse_off[h]);
+      continue;
+    }
     switch (c.type) {
       case SAF3R_PROBE:
       case SAF3R_SCAN:

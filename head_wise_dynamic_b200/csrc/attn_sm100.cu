@@ -243,8 +243,6 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm,
                                               const CUtensorMap& tmK, const CUtensorMap& tmV,
                                               const CUtensorMap& tmQC, const CUtensorMap& tmKC,
                                               const CUtensorMap& tmVC, int lane) {
-  volatile int* abort = &sm.abort;
-  const long long budget = p.wait_budget;
   if (lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -783,7 +781,17 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
     } else if (qrow < p.N) {
       token = qrow;
     }
-    if (token >= 0) {
+    if (hp.part_o != nullptr) {
+      // a token-wise head's patch query against its special keys only: the partial result
+      const int view = token / p.V, slot = token - view * p.V;
+      if (token >= 0 && slot >= p.ns) {
+        const long long a = static_cast<long long>(view) * p.P + (slot - p.ns);
+        float4* dst = reinterpret_cast<float4*>(hp.part_o + a * kD);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        hp.part_lse[a] = den > 0.f ? mmax + log2f(den) : -INFINITY;
+      }
+    } else if (token >= 0) {
       const long long rowoff = (static_cast<long long>(hp.head) * p.N + token) * kD;
       if (p.out_fp32) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + rowoff);

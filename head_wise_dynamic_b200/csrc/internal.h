@@ -88,6 +88,12 @@ struct HeadPlan {
   int32_t nb_base;    // position heads: derived row where the cell-major neighbour rows start
   int32_t lat_stride; // hybrid heads: lattice keys inside a kept tile are counted in the derived run
   int32_t lat_phase;  //   (so the tile runs mask them); 0 = no lattice mask
+  // Non-null: the patch queries of a token-wise head against its special keys only.  The epilogue
+  // then writes, per patch query row a = s*P + patch, the output normalised over those keys
+  // (part_o, fp32 [S*P][64]) and log2 of its softmax denominator in the kernel's scaled-logit units
+  // (part_lse, [S*P]) instead of `out`; the token-wise kernel adds the per-frame keys and merges.
+  float* part_o;
+  float* part_lse;
 };
 
 struct AttnParams {
@@ -124,6 +130,10 @@ struct TokenAttnParams {
   const int32_t* cache;
   const int* ok_flag;
   int* err;
+  // per token-wise head: non-null when its patch queries' special keys ran in the tensor-core
+  // kernel (see HeadPlan::part_o); the kernel then walks only the per-frame lists and merges
+  const float* part_o[kMaxHeads];
+  const float* part_lse[kMaxHeads];
 };
 
 // Tensor-core cosines of the token-wise selection (token_sim.cu): scores[r][c] (fp16, row
