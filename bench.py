@@ -38,10 +38,10 @@ L2_NOTE = "inputs larger than L2 (Q/K/V 3 x 281 MB per call)"
 
 # DRAM traffic of one attention launch on this workload, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum of one S=100-view layer call, one launch, a
-# 1-pass metric set; profiles/attn_sm100_s100_dram.md), valid only for the kernel source it was
+# 1-pass metric set; its summary is kept under profiles/), valid only for the kernel source it was
 # taken on: a changed kernel reports null until it is re-captured.
-ATTN_TRAFFIC = {"kernel_source_sha256": "8a3e7a5a9a5b8aec2e0b0f2611aebf447492138bd3fcf39fb73328ce603aa400",
-                "bytes_per_launch": 618848256 + 265734912, "workload": "s100"}
+ATTN_TRAFFIC = {"kernel_source_sha256": "882784baca5b27d4d158701d7f6769c1f6250c4c3db98b291092a041b4ab4965",
+                "bytes_per_launch": 607632640 + 263734272, "workload": "s100"}
 
 
 def kernel_source_sha256():
