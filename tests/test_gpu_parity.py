@@ -362,6 +362,21 @@ def test_token_heads_tied_features(n_feat):
     check_rows(case, heads, sels, out, lambda h: np.arange(L.N))
 
 
+def test_token_heads_with_and_without_a_partial_plan():
+    """62 heads, 6 of them token-wise: the tensor-core kernel's plan array (64) holds the 62 heads'
+    plans and the partial plans of only the first 2 token heads, so those 2 take their patch queries'
+    special keys on the tensor cores and merge, while the other 4 take them in the gather kernel.
+    Every row of every head against the oracle."""
+    heads = [HeadCfg(SCAN, stride=4, phase=h % 4) for h in range(56)] + \
+            [HeadCfg(TOKEN, k=4), HeadCfg(TOKEN, k=9)] * 3
+    case = Case(_custom(4, 10, heads, seed=95))
+    att, out = run_gpu(case, heads)
+    sel = oracle_select(case, heads)
+    sels = check_selection(case, heads, att, sel)
+    _check_token_heads(case, heads, att, sels, lambda h: np.arange(case.L.N))
+    check_rows(case, heads, sels, out, lambda h: np.arange(case.L.N))
+
+
 def test_s32_token_heads_sampled_rows(s32):
     """Per-frame Top-16 token-wise heads on the S=32 layer (the other heads as configured)."""
     heads = [HeadCfg(TOKEN, k=16)] * 4 + list(s32.wl.heads[4:])
