@@ -556,14 +556,11 @@ __device__ __forceinline__ bool softmax_half(const AttnParams& p, AttnSmem& sm, 
   }
   float s[64];
   {
-    uint32_t raw[2][32];
-    tmem_ld32(tS, raw[0]);
-    tmem_ld32(tS + 32, raw[1]);
+    uint32_t raw[64];
+    tmem_ld64(tS, raw);
     tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[c][i]);
+    for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(raw[i]);
   }
   if (valid != ~0ull) {
 #pragma unroll
