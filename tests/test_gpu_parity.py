@@ -310,6 +310,34 @@ TOKEN_CASES = {
 }
 
 
+@pytest.mark.parametrize("which", ["probe", "tile", "token"])
+def test_out_of_range_cached_index_is_reported(tiny, which):
+    """A cached index that points outside the layer (a probe key past N, a ranked tile past T, a
+    per-frame patch past P) is range-checked where it is consumed: the call records
+    SAF3R_ERR_INDEX, reads nothing out of range, and the next check finds the error word cleared.
+    The cache header's hash covers the layout and the configuration, not the lists, so the planted
+    value gets past the cache check."""
+    hw = _hw()
+    case = tiny if which != "token" else Case(TOKEN_CASES["token_mixed"])
+    heads = case.wl.heads
+    h, kind, bad = {"probe": (1, PROBE, case.L.N + 7), "tile": (2, CORR, case.L.T + 5),
+                    "token": (0, TOKEN, case.L.P + 3)}[which]
+    assert heads[h].kind == kind
+    att, _ = run_gpu(case, heads)
+    lst = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).ravel().astype(np.int32)
+    words = att.cache.view(torch.int32).cpu().numpy().copy()
+    starts = [i for i in np.flatnonzero(words[:len(words) - len(lst) + 1] == lst[0])
+              if np.array_equal(words[i:i + len(lst)], lst)]
+    assert len(starts) == 1, "the exported list is not one contiguous run of the cache"
+    words[starts[0] + len(lst) // 2] = bad
+    att.cache.copy_(torch.from_numpy(words).view(torch.uint8).to(att.cache.device))
+    att(case.q, case.k, case.v)
+    with pytest.raises(hw.Saf3rError) as e:
+        hw.saf3r_check()
+    assert e.value.status == hw.ERR_INDEX
+    hw.saf3r_check()  # the error word was cleared
+
+
 def _check_token_heads(case, heads, att, sels, rows):
     """Per-frame lists of every token-wise head (the given query rows) against the oracle; each
     head is added to `sels`.  Returns {head: lists identical}."""
