@@ -96,6 +96,19 @@ bool make_map_3d(CUtensorMap* m, const void* base, long long rows, int H) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows][64] bf16 with a box of one row: the map of TMA row gathers (four rows per load)
+bool make_map_rows(CUtensorMap* m, const void* base, long long rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows < 1 ? 1 : rows)};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_2d(CUtensorMap* m, const void* base, long long rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
@@ -187,8 +200,28 @@ struct CacheLayout {
   int order_off = 0;
   int tok_kmax = 0;        // token-wise heads: widest per-frame budget
   long long tok_off = 0;   // int32 offset of the per-frame lists [S*P][S][tok_kmax]
+  long long tperm_off = -1;  // token-wise heads on the tensor cores: patch query order [S*P] (-1: none)
+  int n_tg = 0;              // their union groups, one per distinct per-frame budget
+  TokTileGroup tg[kMaxHeads];
+  int tg_of[kMaxHeads];      // per head: its group, or -1
   size_t bytes = 0;
 };
+
+// Token-wise heads run on the tensor cores when the union builder fits the layout and the
+// unions' worst-case storage stays bounded (else the gather kernel takes their patch queries).
+constexpr long long kTokTileMaxEntries = 1ll << 28;  // union entries over all items of a group
+
+bool tok_tiles_on(const Dims& d, const saf3r_head_cfg* cfg) {
+  if (!tok_tiles_fit(d.P)) return false;
+  const long long items = (static_cast<long long>(d.S) * d.P + kItemRows - 1) / kItemRows;
+  bool any = false;
+  for (int h = 0; h < d.H; ++h) {
+    if (cfg[h].type != SAF3R_TOKEN) continue;
+    any = true;
+    if (items * tok_tile_ucap(d.S, d.P, cfg[h].k) > kTokTileMaxEntries) return false;
+  }
+  return any;
+}
 
 CacheLayout cache_layout(const Dims& d, const saf3r_head_cfg* cfg) {
   CacheLayout c;
@@ -209,6 +242,33 @@ CacheLayout cache_layout(const Dims& d, const saf3r_head_cfg* cfg) {
   ints = (ints + 63) & ~size_t(63);
   c.tok_off = static_cast<long long>(ints);
   ints += static_cast<size_t>(d.S) * d.P * d.S * c.tok_kmax;
+  for (int h = 0; h < d.H; ++h) c.tg_of[h] = -1;
+  if (tok_tiles_on(d, cfg)) {
+    const size_t items = (static_cast<size_t>(d.S) * d.P + kItemRows - 1) / kItemRows;
+    ints = (ints + 63) & ~size_t(63);
+    c.tperm_off = static_cast<long long>(ints);
+    ints += static_cast<size_t>(d.S) * d.P;
+    for (int h = 0; h < d.H; ++h) {
+      if (cfg[h].type != SAF3R_TOKEN) continue;
+      int g = 0;
+      while (g < c.n_tg && c.tg[g].k != cfg[h].k) ++g;
+      if (g == c.n_tg) {
+        TokTileGroup& t = c.tg[c.n_tg++];
+        t.k = cfg[h].k;
+        t.ucap = tok_tile_ucap(d.S, d.P, t.k);
+        ints = (ints + 63) & ~size_t(63);
+        t.tn_off = static_cast<long long>(ints);
+        ints += items;
+        ints = (ints + 63) & ~size_t(63);
+        t.tu_off = static_cast<long long>(ints);
+        ints += items * t.ucap;
+        ints = (ints + 63) & ~size_t(63);
+        t.tm_off = static_cast<long long>(ints);
+        ints += items * (t.ucap / 64) * kItemRows * 2;
+      }
+      c.tg_of[h] = g;
+    }
+  }
   c.bytes = align256(ints * 4);
   return c;
 }
@@ -218,14 +278,14 @@ struct SparseLayout {
   size_t ok_off = 0, kc_off = 0, vc_off = 0, qc_off = 0, offl_off = 0, seg_off = 0, cnt_off = 0, total = 0;
   long long kc_rows = 0, qc_rows = 0, seg_total = 0, cnt_total = 0;
   int off_total = 0;
-  std::vector<int> kc_begin, n_rows, qc_begin, n_lat, n_off, off_list;
-  // token-wise heads whose patch queries' special keys run in the tensor-core kernel (one extra
-  // plan each, while the plans fit), with their partial outputs in the workspace
-  std::vector<int> use_part;
-  std::vector<size_t> part_o_off, part_lse_off;
+  std::vector<int> kc_begin, n_rows, qc_begin, n_q, n_lat, n_off, off_list;
+  // token-wise heads whose patch queries run in the tensor-core kernel (one extra plan each, while
+  // the plans fit; the gather kernel takes the others)
+  std::vector<int> use_tile;
   // shared plan lists
   struct List {
     int kind, param, tail, cap, n_items;  // tail: rows of the derived run that ends every item (tile lists)
+    int grp;                              // token-wise lists: the union group
     long long seg_begin, cnt_begin;
   };
   std::vector<List> lists;
@@ -246,20 +306,20 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
   s.kc_begin.assign(H, 0);
   s.n_rows.assign(H, 0);
   s.qc_begin.assign(H, -1);
+  s.n_q.assign(H, 0);
   s.n_lat.assign(H, 0);
   s.n_off.assign(H, 0);
   s.off_list.assign(H, 0);
   s.list_of.assign(H, -1);
-  s.use_part.assign(H, 0);
-  s.part_o_off.assign(H, 0);
-  s.part_lse_off.assign(H, 0);
+  s.use_tile.assign(H, 0);
   const int nsp = d.ns * d.S;
-  {
+  const CacheLayout cl = cache_layout(d, cfg);
+  if (cl.tperm_off >= 0) {
     int plans = 0;  // plans of the tensor-core kernel without the extra ones
     for (int h = 0; h < H; ++h) plans += cfg[h].type != SAF3R_TOKEN || nsp > 0;
     for (int h = 0; h < H; ++h)
-      if (cfg[h].type == SAF3R_TOKEN && nsp > 0 && plans < kMaxHeads) {
-        s.use_part[h] = 1;
+      if (cfg[h].type == SAF3R_TOKEN && plans < kMaxHeads) {
+        s.use_tile[h] = 1;
         ++plans;
       }
   }
@@ -270,18 +330,21 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
       case SAF3R_POSITION:
         rows = nsp + d.P + d.P * (d.S - 1);
         s.qc_begin[h] = static_cast<int>(s.qc_rows);
+        s.n_q[h] = d.N;
         s.qc_rows += d.N;
         break;
       case SAF3R_PROBE:
         rows = nsp + c.k;
         break;
-      case SAF3R_TOKEN:  // the special-token queries, gathered for the tensor-core kernel, and
-                         // the special keys of the patch queries' partial plan
-        if (nsp > 0) {
+      case SAF3R_TOKEN:  // the special-token queries, gathered for the tensor-core kernel; with a
+                         // tensor-core plan for the patch queries, also those (in the cached order)
+                         // and the special keys
+        s.n_q[h] = nsp + (s.use_tile[h] ? d.S * d.P : 0);
+        if (s.n_q[h] > 0) {
           s.qc_begin[h] = static_cast<int>(s.qc_rows);
-          s.qc_rows += nsp;
+          s.qc_rows += s.n_q[h];
         }
-        if (s.use_part[h]) rows = nsp;
+        if (s.use_tile[h]) rows = nsp;
         break;
       case SAF3R_SCAN:
       case SAF3R_HYBRID: {  // the lattice, then the specials off it
@@ -305,6 +368,28 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
     s.kc_begin[h] = static_cast<int>(s.kc_rows);
     s.n_rows[h] = rows;
     s.kc_rows += rows;
+    if (s.use_tile[h]) {
+      const int g = cl.tg_of[h];
+      int found = -1;
+      for (size_t i = 0; i < s.lists.size(); ++i)
+        if (s.lists[i].kind == SAF3R_TOKEN && s.lists[i].grp == g) found = static_cast<int>(i);
+      if (found < 0) {
+        SparseLayout::List l;
+        l.kind = SAF3R_TOKEN;
+        l.param = c.k;
+        l.tail = nsp;
+        l.grp = g;
+        l.n_items = items_of(d.S * d.P);
+        l.cap = 2;
+        l.seg_begin = s.seg_total;
+        l.cnt_begin = s.cnt_total;
+        s.seg_total += static_cast<long long>(l.cap) * l.n_items;
+        s.cnt_total += 2 * l.n_items;
+        s.lists.push_back(l);
+        found = static_cast<int>(s.lists.size()) - 1;
+      }
+      s.list_of[h] = found;
+    }
     if (c.type == SAF3R_POSITION || tile_kind(c.type)) {
       // tile heads share a list when their budget and derived-run length agree (the lattice
       // masks of a hybrid head are applied in the kernel, not stored in the list)
@@ -320,6 +405,7 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
         l.kind = kind;
         l.param = param;
         l.tail = tail;
+        l.grp = -1;
         l.n_items = c.type == SAF3R_POSITION ? items_of(d.N) : (d.T + 3) / 4;
         l.cap = c.type == SAF3R_POSITION ? position_cap(d, c.radius) : 4 * c.k + 1;
         l.seg_begin = s.seg_total;
@@ -346,14 +432,6 @@ SparseLayout sparse_layout(const Dims& d, const saf3r_head_cfg* cfg) {
   off = align256(off + static_cast<size_t>(s.seg_total) * sizeof(Seg));
   s.cnt_off = off;
   off = align256(off + static_cast<size_t>(s.cnt_total) * 4);
-  for (int h = 0; h < H; ++h) {
-    if (!s.use_part[h]) continue;
-    const size_t rows = static_cast<size_t>(d.S) * d.P;
-    s.part_o_off[h] = off;
-    off = align256(off + rows * kD * sizeof(float));
-    s.part_lse_off[h] = off;
-    off = align256(off + rows * sizeof(float));
-  }
   s.total = off;
   return s;
 }
@@ -370,6 +448,9 @@ double est_keys(const Dims& d, const saf3r_head_cfg& c, const SparseLayout& s, i
       return 1.5 * kTile * c.k + d.ns * d.S;
     case SAF3R_HYBRID:
       return 1.5 * kTile * c.k + s.n_rows[h];
+    case SAF3R_TOKEN:  // the patch queries' plan: the specials, then about twelve times the
+                       // per-frame budget per frame in an item's union
+      return d.ns * d.S + 12.0 * d.S * c.k;
     default:
       return d.N;
   }
@@ -414,6 +495,7 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   DerivedArgs da;
   std::memset(&da, 0, sizeof(da));
   da.S = d.S; da.V = d.V; da.ns = d.ns; da.P = d.P; da.N = d.N;
+  da.tperm_off = cl.tperm_off;
   bool any_scan = false;
   for (int h = 0; h < d.H; ++h) {
     if (s.n_rows[h] == 0 && s.qc_begin[h] < 0) continue;
@@ -423,6 +505,7 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     x.kc_begin = s.kc_begin[h];
     x.n_rows = s.n_rows[h];
     x.qc_begin = s.qc_begin[h];
+    x.n_q = s.n_q[h];
     x.stride = cfg[h].stride;
     x.phase = cfg[h].phase;
     x.n_lat = s.n_lat[h];
@@ -443,6 +526,10 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     if (l.kind == SAF3R_POSITION) {
       st = cuda_status(launch_plan_position(l.n_items, d.S, d.gh, d.gw, d.ns, d.N, l.param, l.cap,
                                             segs + l.seg_begin, cnts + l.cnt_begin, stream));
+    } else if (l.kind == SAF3R_TOKEN) {
+      const TokTileGroup& g = cl.tg[l.grp];
+      st = cuda_status(launch_plan_token(cache_i + g.tn_off, g.ucap, l.n_items, l.tail, segs + l.seg_begin,
+                                         cnts + l.cnt_begin, dev.err, stream));
     } else {
       st = cuda_status(launch_plan_corr(cache_i + cl.corr_off, cache_i + cl.order_off, cl.corr_kmax, l.param, d.T,
                                         d.N, d.V, d.ns, l.tail, segs + l.seg_begin, l.cap, cnts + l.cnt_begin,
@@ -455,34 +542,35 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   // attention
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
-  // the patch queries of token-wise heads run in their own kernel (no shared key runs) over their
-  // per-frame lists; their special keys (a dense block: every patch query keeps them) run here as
-  // a partial plan merged by that kernel, and their special-token queries (every key: dense rows)
-  // and every other head run here as well
+  // every head runs here; a token-wise head has two plans: its special-token queries (every key:
+  // dense rows) and its patch queries (the cached order, each item over the special keys and
+  // its rows' union of per-frame keys).  A token-wise head whose second plan does not fit the
+  // plan array has its patch queries run in the gather kernel instead
   struct PlanRef {
     int h;
-    bool part;
+    bool part;  // a token-wise head's patch queries
   };
   std::vector<PlanRef> order;
   TokenAttnParams tp;
   std::memset(&tp, 0, sizeof(tp));
+  const int nsp = d.ns * d.S;
   for (int h = 0; h < d.H; ++h) {
     if (cfg[h].type == SAF3R_TOKEN) {
-      tp.heads[tp.n_heads] = h;
-      tp.k[tp.n_heads] = cfg[h].k;
-      if (s.use_part[h]) {
-        tp.part_o[tp.n_heads] = reinterpret_cast<const float*>(ws + s.part_o_off[h]);
-        tp.part_lse[tp.n_heads] = reinterpret_cast<const float*>(ws + s.part_lse_off[h]);
+      if (s.use_tile[h]) {
         order.push_back({h, true});
+      } else {
+        tp.heads[tp.n_heads] = h;
+        tp.k[tp.n_heads] = cfg[h].k;
+        ++tp.n_heads;
       }
-      ++tp.n_heads;
-      if (s.qc_begin[h] >= 0) order.push_back({h, false});
+      if (nsp > 0) order.push_back({h, false});
     } else {
       order.push_back({h, false});
     }
   }
-  const int nsp = d.ns * d.S;
-  auto plan_keys = [&](const PlanRef& r) { return r.part ? static_cast<double>(nsp) : est_keys(d, cfg[r.h], s, r.h); };
+  auto plan_keys = [&](const PlanRef& r) {
+    return (cfg[r.h].type == SAF3R_TOKEN && !r.part) ? static_cast<double>(d.N) : est_keys(d, cfg[r.h], s, r.h);
+  };
   std::stable_sort(order.begin(), order.end(),
                    [&](const PlanRef& a, const PlanRef& b) { return plan_keys(a) > plan_keys(b); });
   const int n_main = static_cast<int>(order.size());
@@ -494,12 +582,13 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     HeadPlan& hp = p.heads[i];
     hp.head = h;
     hp.kind = c.type;
-    hp.q_src = part ? 0 : (c.type == SAF3R_POSITION ? 1 : (tile_kind(c.type) ? 2 : (c.type == SAF3R_TOKEN ? 3 : 0)));
-    hp.q_base = part ? 0 : (tile_kind(c.type) ? cl.order_off : (s.qc_begin[h] < 0 ? 0 : s.qc_begin[h]));
+    hp.q_src = part ? 4 : (c.type == SAF3R_POSITION ? 1 : (tile_kind(c.type) ? 2 : (c.type == SAF3R_TOKEN ? 3 : 0)));
+    hp.q_base = part ? s.qc_begin[h] + nsp
+                     : (tile_kind(c.type) ? cl.order_off : (s.qc_begin[h] < 0 ? 0 : s.qc_begin[h]));
     hp.lat_stride = c.type == SAF3R_HYBRID ? c.stride : 0;
     hp.lat_phase = c.type == SAF3R_HYBRID ? c.phase : 0;
     hp.kc_base = s.kc_begin[h];
-    hp.n_items = (c.type == SAF3R_TOKEN && !part) ? items_of(d.ns * d.S) : items_of(d.N);
+    hp.n_items = c.type == SAF3R_TOKEN ? items_of(part ? d.S * d.P : nsp) : items_of(d.N);
     hp.item_begin = item;
     item += hp.n_items;
     hp.seg_list = -1;
@@ -507,14 +596,18 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
     hp.cnt_list = 0;
     hp.radius = c.radius;
     hp.nb_base = d.ns * d.S + d.P;
-    hp.part_o = nullptr;
-    hp.part_lse = nullptr;
+    hp.glist = nullptr;
+    hp.gmask = nullptr;
     if (part) {
-      // every query row against the head's derived special rows; the patch rows' results go to
-      // the partial buffers
-      hp.seg = Seg{1, 0, nsp, kSegAllQuarters};
-      hp.part_o = reinterpret_cast<float*>(ws + s.part_o_off[h]);
-      hp.part_lse = reinterpret_cast<float*>(ws + s.part_lse_off[h]);
+      // per item: the head's derived special rows, then the union of its rows' per-frame keys
+      const TokTileGroup& g = cl.tg[cl.tg_of[h]];
+      const auto& l = s.lists[s.list_of[h]];
+      hp.seg_list = static_cast<int>(l.seg_begin);
+      hp.seg_cap = l.cap;
+      hp.cnt_list = static_cast<int>(l.cnt_begin);
+      hp.seg = Seg{0, 0, 0, 0};
+      hp.glist = cache_i + g.tu_off;
+      hp.gmask = reinterpret_cast<const uint64_t*>(cache_i + g.tm_off);
       continue;
     }
     switch (c.type) {
@@ -549,11 +642,14 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   p.wait_budget = t_wait_budget;
   p.withhold_arrive = t_withhold_arrive ? 1 : 0;
   t_withhold_arrive = false;
+  p.tok_perm = cl.tperm_off >= 0 && cache_i ? cache_i + cl.tperm_off : nullptr;
 
   if (t_ev_start && t_ev_stop && cudaEventRecord(t_ev_start, stream) != cudaSuccess) return SAF3R_ERR_CUDA;
   if (n_main > 0) {
-    CUtensorMap tq, tk, tv, tqc, tkc, tvc;
-    if (!make_map_3d(&tq, q, d.N, d.H) || !make_map_3d(&tk, k, d.N, d.H) || !make_map_3d(&tv, v, d.N, d.H))
+    CUtensorMap tq, tk, tv, tqc, tkc, tvc, tkg, tvg;
+    if (!make_map_3d(&tq, q, d.N, d.H) || !make_map_3d(&tk, k, d.N, d.H) || !make_map_3d(&tv, v, d.N, d.H) ||
+        !make_map_rows(&tkg, k, static_cast<long long>(d.H) * d.N) ||
+        !make_map_rows(&tvg, v, static_cast<long long>(d.H) * d.N))
       return SAF3R_ERR_CUDA;
     const void* kc_base = s.kc_rows > 0 ? static_cast<const void*>(kc) : k;
     const void* vc_base = s.kc_rows > 0 ? static_cast<const void*>(vc) : v;
@@ -562,7 +658,7 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
         !make_map_2d(&tvc, vc_base, s.kc_rows > 0 ? s.kc_rows : 1) ||
         !make_map_2d(&tqc, qc_base, s.qc_rows > 0 ? s.qc_rows : 1))
       return SAF3R_ERR_CUDA;
-    st = cuda_status(launch_attention(p, tq, tk, tv, tqc, tkc, tvc, dev.sms, stream));
+    st = cuda_status(launch_attention(p, tq, tk, tv, tqc, tkc, tvc, tkg, tvg, dev.sms, stream));
     ++launches;
     if (st != SAF3R_OK) return st;
   }
@@ -661,7 +757,8 @@ size_t saf3r_workspace_bytes(const saf3r_layout* L, const saf3r_head_cfg* cfg, i
       corr |= tile_kind(cfg[h].type);
       tok |= cfg[h].type == SAF3R_TOKEN;
     }
-    return select_workspace_bytes(n_probe, d.N, d.T, d.dino_dim, corr, tok ? static_cast<long long>(d.S) * d.P : 0);
+    return select_workspace_bytes(n_probe, d.N, d.T, d.dino_dim, corr, tok ? static_cast<long long>(d.S) * d.P : 0,
+                                  cache_layout(d, cfg).tperm_off >= 0 ? d.P : 0);
   }
   if (op == SAF3R_OP_SPARSE) return sparse_layout(d, cfg).total;
   return 0;
@@ -699,6 +796,9 @@ saf3r_status saf3r_select_kv(const saf3r_layout* L, const saf3r_head_cfg* cfg, c
   sp.S = d.S;
   sp.tok_kmax = cl.tok_kmax;
   sp.tok_off = cl.tok_off;
+  sp.tperm_off = cl.tperm_off;
+  sp.n_tg = cl.n_tg;
+  for (int g = 0; g < cl.n_tg; ++g) sp.tg[g] = cl.tg[g];
   sp.num_sms = dev.sms;
   sp.err = dev.err;
   sp.wait_budget = t_wait_budget;

@@ -14,8 +14,15 @@
 // counted, a cell outside its neighbourhood, the ragged end of a run) are
 // masked to -inf in its softmax.
 //
+// Token-wise heads' patch queries (q_src 4) come in a cached order that makes queries with the
+// same best matches neighbours; each item streams the head's special keys (derived rows) and then
+// the union of its rows' per-frame keys, whose K/V rows arrive by TMA row gathers (four listed
+// rows per instruction, 16 lanes of the producer warp), and every row keeps its own keys of that
+// union through a cached bitmask.
+//
 // Warp roles (12 warps, three warpgroups):
-//   warp 0      TMA producer: Q tiles, then K and V blocks into a 4-stage ring
+//   warp 0      TMA producer: Q tiles, then K and V blocks into a 4-stage ring (for gathered
+//               runs 16 lanes issue the row gathers)
 //   warp 1      MMA issuer: O_t += P_t V, then S_t = Q_t K^T of the next block (the whole warp
 //               waits and computes descriptors, one elected lane issues)
 //   warps 2-3   idle (their registers go to the softmax warpgroups)
@@ -234,6 +241,90 @@ __device__ __forceinline__ bool producer_item(const AttnParams& p, AttnSmem& sm,
   return true;
 }
 
+// Rows 4l..4l+3 of a gathered half (src 2) for lane l < 16, as rows of the [H*N][64] K/V maps.
+// Rows past the half's count, of an absent half, or whose listed token is out of range
+// (reported) load the head's token 0 instead: an in-range row whose keys every row masks.
+__device__ __forceinline__ int4 gather_rows(const AttnParams& p, const HeadPlan& hp, const Half& h, int lane) {
+  const int pad = hp.head * p.N;
+  int r[4] = {pad, pad, pad, pad};
+  const int b = 4 * lane;
+  if (lane < 16 && h.have && h.s.src == 2 && b < h.cnt) {
+    const int4 t4 = *reinterpret_cast<const int4*>(hp.glist + h.s.row0 + h.off + b);
+    const int t[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (b + i >= h.cnt) continue;
+      if (t[i] >= 0 && t[i] < p.N)
+        r[i] = hp.head * p.N + t[i];
+      else
+        atomicCAS(p.err, 0, SAF3R_ERR_INDEX);
+    }
+  }
+  return make_int4(r[0], r[1], r[2], r[3]);
+}
+
+// One 64-row half of a K or V stage: derived rows by one TMA box (lane 0), else (gathered rows,
+// or an absent half) four rows per lane of lanes 0-15 by TMA row gathers.
+__device__ __forceinline__ void load_half_gathered(const HeadPlan& hp, const Half& h, const int4& rows,
+                                                   uint8_t* dst, const CUtensorMap& m2, const CUtensorMap& mg,
+                                                   uint64_t* bar, int lane) {
+  if (h.have && h.s.src == 1) {
+    if (lane == 0) tma_load_2d(dst, &m2, 0, hp.kc_base + h.s.row0 + h.off, bar);
+  } else if (lane < 16) {
+    tma_gather4(dst + lane * 512, &mg, 0, rows.x, rows.y, rows.z, rows.w, bar);
+  }
+}
+
+// One item of a token-wise head's patch queries, run by the whole producer warp: derived Q rows
+// and the derived special K/V rows as TMA boxes, the union's K/V rows as TMA row gathers (each
+// full stage barrier expects one whole tile, as for the other heads).
+__device__ __forceinline__ bool producer_item_gather(const AttnParams& p, AttnSmem& sm, const CUtensorMap& tmQC,
+                                                     const CUtensorMap& tmKC, const CUtensorMap& tmVC,
+                                                     const CUtensorMap& tmKG, const CUtensorMap& tmVG,
+                                                     ItemInfo& it, const HeadPlan& hp, uint32_t& k_issued,
+                                                     uint32_t& v_issued, uint32_t& q_issued, int lane) {
+  volatile int* abort = &sm.abort;
+  const long long budget = p.wait_budget;
+  if (q_issued > 0 &&
+      !__all_sync(0xffffffffu, mbar_wait(&sm.q_empty, (q_issued - 1) & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)))
+    return false;
+  if (lane == 0) {
+    mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
+    for (int quarter = 0; quarter < 4; ++quarter)
+      tma_load_2d(sm.q[quarter >> 1] + (quarter & 1) * kHalfBytes, &tmQC, 0, hp.q_base + it.q0 + quarter * 64,
+                  &sm.q_full);
+  }
+  ++q_issued;
+  for (int b = 0; b < it.nblk; ++b) {
+    const Half h0 = it.w.next();
+    const Half h1 = it.w.next();
+    const int4 r0 = gather_rows(p, hp, h0, lane), r1 = gather_rows(p, hp, h1, lane);
+    const uint32_t stage = k_issued % kStages, ph = (k_issued / kStages) & 1;
+    if (k_issued >= kStages &&
+        !__all_sync(0xffffffffu, mbar_wait(&sm.k_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)))
+      return false;
+    if (lane == 0) mbar_arrive_expect_tx(&sm.k_full[stage], kTileBytes);
+    __syncwarp();
+    load_half_gathered(hp, h0, r0, sm.k[stage], tmKC, tmKG, &sm.k_full[stage], lane);
+    load_half_gathered(hp, h1, r1, sm.k[stage] + kHalfBytes, tmKC, tmKG, &sm.k_full[stage], lane);
+    ++k_issued;
+    if (v_issued >= kStages &&
+        !__all_sync(0xffffffffu, mbar_wait(&sm.v_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)))
+      return false;
+    if (lane == 0) {
+      // the block's halves for the softmax warps; the arrival below releases them with the stage
+      sm.info[stage][0] = h0;
+      sm.info[stage][1] = h1;
+      mbar_arrive_expect_tx(&sm.v_full[stage], kTileBytes);
+    }
+    __syncwarp();
+    load_half_gathered(hp, h0, r0, sm.v[stage], tmVC, tmVG, &sm.v_full[stage], lane);
+    load_half_gathered(hp, h1, r1, sm.v[stage] + kHalfBytes, tmVC, tmVG, &sm.v_full[stage], lane);
+    ++v_issued;
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------ TMA producer (one warp, lane 0 issues)
 //
 // At each item the whole warp copies the item's key runs into shared memory (a list head's runs
@@ -242,7 +333,8 @@ __device__ __forceinline__ bool producer_item(const AttnParams& p, AttnSmem& sm,
 __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm, const CUtensorMap& tmQ,
                                               const CUtensorMap& tmK, const CUtensorMap& tmV,
                                               const CUtensorMap& tmQC, const CUtensorMap& tmKC,
-                                              const CUtensorMap& tmVC, int lane) {
+                                              const CUtensorMap& tmVC, const CUtensorMap& tmKG,
+                                              const CUtensorMap& tmVG, int lane) {
   if (lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -258,8 +350,16 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm,
       it.w.list = sm.segbuf;
     }
     __syncwarp();
-    if (lane == 0) ok = producer_item(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, it, hp, k_issued, v_issued, q_issued);
-    ok = __shfl_sync(0xffffffffu, ok, 0);  // the runs are not overwritten before lane 0 has walked them
+    if (hp.q_src == 4) {
+      ok = producer_item_gather(p, sm, tmQC, tmKC, tmVC, tmKG, tmVG, it, hp, k_issued, v_issued, q_issued, lane);
+      __syncwarp();
+    } else {
+      if (lane == 0) ok = producer_item(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, it, hp, k_issued, v_issued, q_issued);
+      ok = __shfl_sync(0xffffffffu, ok, 0);  // the runs are not overwritten before lane 0 has walked them
+      k_issued = __shfl_sync(0xffffffffu, k_issued, 0);
+      v_issued = __shfl_sync(0xffffffffu, v_issued, 0);
+      q_issued = __shfl_sync(0xffffffffu, q_issued, 0);
+    }
   }
   if (lane != 0) return;
   // Teardown: every copy lane 0 issued must have landed before the CTA exits
@@ -403,7 +503,9 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, AttnSmem& sm, uint
 //   kMaskTiles     - + tiles this row's quarter does not keep, special tokens already
 //                    counted inside a tile (correspondence heads)
 //   kMaskCells     - + neighbour cells of this row's grid cell (position heads)
-constexpr int kMaskPlain = 0, kMaskTiles = 1, kMaskCells = 2;
+//   kMaskBits      - the row's cached bitmask over the item's union (token-wise patch queries;
+//                    computed by softmax_blocks_bits, which passes it in)
+constexpr int kMaskPlain = 0, kMaskTiles = 1, kMaskCells = 2, kMaskBits = 3;
 constexpr int kNbIntervals = 2 * kMaxRadius + 1;
 
 struct RowCtx {
@@ -413,6 +515,7 @@ struct RowCtx {
   uint32_t lane_off; // TMEM lane field of this warp
   int nb_lo[2][kNbIntervals], nb_hi[2][kNbIntervals];  // position heads: kept derived rows [lo, hi) per tile
   int lat_stride, lat_phase;  // hybrid heads: the lattice (counted in the derived run), 0 = none
+  const uint64_t* gmask;      // token-wise patch queries: [half-block of the union][item row] bitmasks
   bool withhold;     // test hook: skip the next P-ready arrival (the MMA warp's wait then runs out)
 };
 
@@ -670,6 +773,45 @@ __device__ __forceinline__ bool softmax_blocks(const AttnParams& p, AttnSmem& sm
   return true;
 }
 
+// All key blocks of one item of a token-wise head's patch queries.  Its runs are the derived
+// special rows, then its union: half-block i of the item is a special one for i < nsh (every row
+// keeps those keys), else union half-block i - nsh, whose mask words (one per item row) sit at a
+// known place, so this thread loads its words for the next block while the current one runs.
+__device__ __forceinline__ bool softmax_blocks_bits(const AttnParams& p, AttnSmem& sm, SoftmaxState& ss,
+                                                    uint32_t tmem, ItemInfo& it, RowCtx& rc, float (&m)[2],
+                                                    float (&l)[2]) {
+  const Seg sp = it.w.list[0], un = it.w.list[1];
+  const int nsh = (sp.len + 63) >> 6, nuh = (un.len + 63) >> 6;
+  const uint64_t* gm = rc.gmask + static_cast<long long>(un.row0 >> 6) * kItemRows + rc.r;
+  auto words = [&](int j, uint64_t& w0, uint64_t& w1) {
+    const int u = 2 * j + rc.kh - nsh;
+    if (u >= 0 && u < nuh) {
+      w0 = gm[static_cast<long long>(u) * kItemRows];
+      w1 = gm[static_cast<long long>(u) * kItemRows + 128];
+    } else {
+      w0 = w1 = ~0ull;
+    }
+  };
+  uint64_t c0, c1;
+  words(0, c0, c1);
+  for (int j = 0; j < it.nblk; ++j) {
+    uint64_t n0 = ~0ull, n1 = ~0ull;
+    if (j + 1 < it.nblk) words(j + 1, n0, n1);
+    const uint32_t c = ss.kv_c + j, st = c % kStages;
+    if (!__all_sync(0xffffffffu, mbar_wait(&sm.v_full[st], (c / kStages) & 1, &sm.abort, p.err, p.wait_budget,
+                                           SAF3R_ERR_TIMEOUT)))
+      return false;
+    const Half hb = sm.info[st][rc.kh];
+    const uint64_t cnt = !hb.have ? 0ull : (hb.cnt >= 64 ? ~0ull : ((1ull << hb.cnt) - 1ull));
+    if (!softmax_half<kMaskBits>(p, sm, ss, tmem, rc, 0, j, cnt & c0, m[0], l[0])) return false;
+    if (!softmax_half<kMaskBits>(p, sm, ss, tmem, rc, 1, j, cnt & c1, m[1], l[1])) return false;
+    c0 = n0;
+    c1 = n1;
+  }
+  ss.kv_c += it.nblk;
+  return true;
+}
+
 __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, uint32_t tmem, int warp, int lane) {
   volatile int* abort = &sm.abort;
   const long long budget = p.wait_budget;
@@ -689,7 +831,10 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
     const HeadPlan& hp = p.heads[it.hi];
     float m[2] = {-INFINITY, -INFINITY};  // running max of this key half, log2 units, per tile
     float l[2] = {0.f, 0.f};              // running sum of this key half, per tile
-    if (hp.kind == SAF3R_POSITION) {
+    if (hp.q_src == 4) {
+      rc.gmask = hp.gmask;
+      ok = softmax_blocks_bits(p, sm, ss, tmem, it, rc, m, l);
+    } else if (hp.kind == SAF3R_POSITION) {
       // neighbour cells of each tile row's grid cell, as kept derived rows [lo, hi)
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
@@ -775,20 +920,19 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, AttnSmem& sm, 
     } else if (hp.q_src == 2) {
       const int u = mapped_tile(p, hp, it.local, quarter);
       if (u >= 0 && u * 64 + (r & 63) < p.N) token = u * 64 + (r & 63);
+    } else if (hp.q_src == 4) {
+      // a token-wise head's patch query, in the cached order
+      if (qrow < p.P * p.S) {
+        const int u = p.tok_perm[qrow];
+        if (u >= 0 && u < p.P * p.S)
+          token = (u / p.P) * p.V + p.ns + (u % p.P);
+        else
+          atomicCAS(p.err, 0, SAF3R_ERR_INDEX);
+      }
     } else if (qrow < p.N) {
       token = qrow;
     }
-    if (hp.part_o != nullptr) {
-      // a token-wise head's patch query against its special keys only: the partial result
-      const int view = token / p.V, slot = token - view * p.V;
-      if (token >= 0 && slot >= p.ns) {
-        const long long a = static_cast<long long>(view) * p.P + (slot - p.ns);
-        float4* dst = reinterpret_cast<float4*>(hp.part_o + a * kD);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        hp.part_lse[a] = den > 0.f ? mmax + log2f(den) : -INFINITY;
-      }
-    } else if (token >= 0) {
+    if (token >= 0) {
       const long long rowoff = (static_cast<long long>(hp.head) * p.N + token) * kD;
       if (p.out_fp32) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + rowoff);
@@ -811,7 +955,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmQC, const __grid_constant__ CUtensorMap tmKC,
-                      const __grid_constant__ CUtensorMap tmVC) {
+                      const __grid_constant__ CUtensorMap tmVC, const __grid_constant__ CUtensorMap tmKG,
+                      const __grid_constant__ CUtensorMap tmVG) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -848,7 +993,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) reg_dealloc_dec<104>();  // 104*128 + 200*256 = 168*384 registers
   if (warp == 0) {
-    producer_role(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, lane);
+    producer_role(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, tmKG, tmVG, lane);
     __syncwarp();
   } else if (warp == 1) {
     mma_role(p, sm, tmem);
@@ -870,14 +1015,15 @@ size_t attn_smem_bytes() { return sizeof(AttnSmem) + 1024; }
 
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmQC, const CUtensorMap& tmKC,
-                             const CUtensorMap& tmVC, int num_sms, cudaStream_t stream) {
+                             const CUtensorMap& tmVC, const CUtensorMap& tmKG, const CUtensorMap& tmVG,
+                             int num_sms, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.total_items < num_sms ? p.total_items : num_sms;
   if (grid <= 0) return cudaSuccess;
-  attn_sm100_kernel<<<grid, kThreads, smem, stream>>>(p, tmQ, tmK, tmV, tmQC, tmKC, tmVC);
+  attn_sm100_kernel<<<grid, kThreads, smem, stream>>>(p, tmQ, tmK, tmV, tmQC, tmKC, tmVC, tmKG, tmVG);
   return cudaGetLastError();
 }
 

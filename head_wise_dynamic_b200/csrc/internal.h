@@ -17,7 +17,7 @@ constexpr uint32_t kCacheMagic = 0x52334653u;  // "SF3R"
 // Teardown waits (copies already issued must land before a CTA exits) have their own fixed
 // budget, independent of the per-call wait budget, so a short test budget cannot cut them off.
 constexpr long long kDrainBudget = 1000000000LL;  // clock cycles (~0.5 s)
-constexpr uint32_t kCacheVersion = 2;
+constexpr uint32_t kCacheVersion = 3;
 
 // Heads whose keys include ranked DINO tiles (they share the cached tile lists), and heads
 // whose keys include the stride lattice (they get the lattice as derived rows).
@@ -58,7 +58,9 @@ constexpr int kCacheHeaderBytes = 512;
 
 // A run of key rows of one head, fed to the attention kernel 64 rows at a time.
 // src 0: the caller's K/V ([H][N][64], row = token); src 1: the head's derived
-// rows in the workspace (row relative to the head's derived base).
+// rows in the workspace (row relative to the head's derived base); src 2: the tokens
+// listed at the head's gathered-key list (entry row0 + i, row0 a multiple of 4), rows gathered
+// from the caller's K/V.
 struct Seg {
   int32_t src;
   int32_t row0;
@@ -69,13 +71,33 @@ struct Seg {
 constexpr uint32_t kSegAllQuarters = 0xFu;
 constexpr uint32_t kSegCellMask = 0x10u;
 
+// Token-wise heads on the tensor cores.  The patch queries are ordered so that queries with
+// the same best matches are neighbours (perm[i] = patch query row s*P + p of row i); each
+// 256-row item then streams the union of its rows' per-frame keys, ascending by token, and
+// every row keeps its own keys of that union through a bitmask.  One group per distinct
+// per-frame budget k; int32 offsets into the cache:
+//   tn_off: [items] union length U of each item
+//   tu_off: [items][ucap] the union's tokens (entries [U, ucap) unused)
+//   tm_off: [items][ucap / 64][256] uint64 masks: bit b of word (item, h, r) = row r keeps
+//           union entry 64 h + b
+struct TokTileGroup {
+  int k;
+  int ucap;  // a multiple of 64, at least every item's union
+  long long tn_off, tu_off, tm_off;
+};
+__host__ __device__ inline int tok_tile_ucap(int S, int P, int k) {
+  const long long per_frame = static_cast<long long>(k) * kItemRows < P ? static_cast<long long>(k) * kItemRows : P;
+  return static_cast<int>((static_cast<long long>(S) * per_frame + 63) / 64 * 64);
+}
+
 // Per-head plan of one attention launch (kernel parameter).
 struct HeadPlan {
   int32_t head;       // head index h in [0, H)
   int32_t kind;       // saf3r_head_type
   int32_t q_src;      // 0: caller Q rows are tokens; 1: derived cell-major Q rows (position heads);
                       // 2: caller Q, each 64-row quarter of an item is the query tile qmap[4*item + quarter];
-                      // 3: derived Q rows of the special tokens only, view by view (token-wise heads)
+                      // 3: derived Q rows of the special tokens only, view by view (token-wise heads);
+                      // 4: derived Q rows of the patch queries in the order perm (token-wise heads)
   int32_t q_base;     // derived Q row base (q_src == 1); qmap offset (q_src == 2)
   int32_t kc_base;    // derived K/V row base
   int32_t n_items;    // work items (256 query rows each)
@@ -88,12 +110,9 @@ struct HeadPlan {
   int32_t nb_base;    // position heads: derived row where the cell-major neighbour rows start
   int32_t lat_stride; // hybrid heads: lattice keys inside a kept tile are counted in the derived run
   int32_t lat_phase;  //   (so the tile runs mask them); 0 = no lattice mask
-  // Non-null: the patch queries of a token-wise head against its special keys only.  The epilogue
-  // then writes, per patch query row a = s*P + patch, the output normalised over those keys
-  // (part_o, fp32 [S*P][64]) and log2 of its softmax denominator in the kernel's scaled-logit units
-  // (part_lse, [S*P]) instead of `out`; the token-wise kernel adds the per-frame keys and merges.
-  float* part_o;
-  float* part_lse;
+  // q_src 4 (token-wise patch queries): the group's union tokens and row masks (see TokTileGroup)
+  const int32_t* glist;
+  const uint64_t* gmask;
 };
 
 struct AttnParams {
@@ -110,6 +129,7 @@ struct AttnParams {
   const int* ok_flag;  // nonzero: cache check passed (NULL: no check)
   long long wait_budget;
   int32_t withhold_arrive;  // test hook: CTA 0's first softmax warp withholds its first P-ready arrival
+  const int32_t* tok_perm;  // patch query order of the token-wise heads (in the cache)
   HeadPlan heads[kMaxHeads];
 };
 
@@ -130,10 +150,6 @@ struct TokenAttnParams {
   const int32_t* cache;
   const int* ok_flag;
   int* err;
-  // per token-wise head: non-null when its patch queries' special keys ran in the tensor-core
-  // kernel (see HeadPlan::part_o); the kernel then walks only the per-frame lists and merges
-  const float* part_o[kMaxHeads];
-  const float* part_lse[kMaxHeads];
 };
 
 // Tensor-core cosines of the token-wise selection (token_sim.cu): scores[r][c] (fp16, row
@@ -160,6 +176,9 @@ struct SelectPlan {
   int S;
   int tok_kmax;             // token-wise heads: widest per-frame budget (0 = none)
   long long tok_off;
+  long long tperm_off;      // token-wise query order [S*P] (-1: no tensor-core token plans)
+  int n_tg;                 // token-wise union groups (one per distinct k)
+  TokTileGroup tg[kMaxHeads];
   int num_sms;
   int* err;                 // device error word (bounded waits of the tensor-core kernels)
   long long wait_budget;
@@ -173,6 +192,7 @@ struct DerivedHead {
   int kc_begin;     // first global derived K/V row
   int n_rows;       // derived K/V rows of this head
   int qc_begin;     // first global derived Q row (position and token-wise heads), -1 if none
+  int n_q;          // derived Q rows of this head
   int stride, phase, n_lat;  // scan heads
   int probe_off;    // cache int32 offset of the probe key list
   int off_list;     // scan heads: int offset of the off-lattice special list in the workspace
@@ -181,6 +201,7 @@ struct DerivedHead {
 struct DerivedArgs {
   int n;                    // heads with derived rows
   int S, V, ns, P, N;
+  long long tperm_off;      // token-wise heads: cache int32 offset of the patch query order
   long long kc_total;       // derived K/V rows
   long long qc_total;       // derived Q rows
   DerivedHead h[kMaxHeads];
@@ -200,8 +221,9 @@ saf3r_status validate_layout_cfg(const saf3r_layout* L, const saf3r_head_cfg* cf
 size_t attn_smem_bytes();
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmQC, const CUtensorMap& tmKC,
-                             const CUtensorMap& tmVC, int num_sms, cudaStream_t stream);
-size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows);
+                             const CUtensorMap& tmVC, const CUtensorMap& tmKG, const CUtensorMap& tmVG,
+                             int num_sms, cudaStream_t stream);
+size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows, int tiles_P);
 size_t token_rank_smem_bytes(int P, int kmax);
 size_t token_sim_smem_bytes();
 cudaError_t launch_token_sim(const TokenSimParams& p, const CUtensorMap& tm, int num_sms, cudaStream_t stream);
@@ -219,6 +241,16 @@ cudaError_t launch_plan_position(int n_items, int S, int gh, int gw, int ns, int
 cudaError_t launch_plan_corr(const int32_t* ranked, const int32_t* order, int kmax, int kt, int T, int N, int V,
                              int ns, int tail_len, Seg* segs, int cap, int* counts, int* err, cudaStream_t stream);
 cudaError_t launch_token_attention(const TokenAttnParams& p, int num_sms, cudaStream_t stream);
+// token-wise heads on the tensor cores (token_tiles.cu): does the union builder fit this layout;
+// its workspace; the index-build launches (query order, then every group's unions and masks);
+// the per-call key runs of every item: the nsp derived special rows, then the item's union
+bool tok_tiles_fit(int P);
+size_t tok_tiles_workspace_bytes(int S, int P);
+cudaError_t launch_tok_tiles(const int32_t* lists, int S, int P, int V, int ns, int tok_kmax, long long tperm_off,
+                             const TokTileGroup* tg, int n_tg, int32_t* cache, uint8_t* ws, int* err,
+                             cudaStream_t stream, int* n_launch);
+cudaError_t launch_plan_token(const int32_t* tn, int ucap, int n_items, int nsp, Seg* segs, int* counts, int* err,
+                              cudaStream_t stream);
 size_t nmse_workspace_bytes(int H);
 cudaError_t launch_nmse(const float* full, const float* sparse, int H, long long per_head, double* part,
                         double* out, cudaStream_t stream);

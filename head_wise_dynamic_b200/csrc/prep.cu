@@ -50,7 +50,7 @@ __device__ __forceinline__ int derived_token(const DerivedArgs& a, const Derived
     case SAF3R_HYBRID:  // the lattice, then the specials off it
       if (r < d.n_lat) return d.phase + r * d.stride;
       return offlists[d.off_list + (r - d.n_lat)];
-    default:  // SAF3R_CORR: the special tokens
+    default:  // SAF3R_CORR, SAF3R_TOKEN: the special tokens
       return special_token(r, a.V, a.ns);
   }
 }
@@ -123,15 +123,27 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(DerivedArgs a, const u
     } else {
       const int row = static_cast<int>(task - a.kc_total);
       int hi = -1;
-      for (int i = 0; i < a.n; ++i) {
-        const int n_q = a.h[i].kind == SAF3R_TOKEN ? a.ns * a.S : a.N;
-        if (a.h[i].qc_begin >= 0 && row >= a.h[i].qc_begin && row < a.h[i].qc_begin + n_q) hi = i;
-      }
+      for (int i = 0; i < a.n; ++i)
+        if (a.h[i].qc_begin >= 0 && row >= a.h[i].qc_begin && row < a.h[i].qc_begin + a.h[i].n_q) hi = i;
       if (hi < 0) continue;
       const DerivedHead& d = a.h[hi];
-      // position heads: every query in cell-major order; token-wise heads: the special tokens
-      const int tok = d.kind == SAF3R_TOKEN ? special_token(row - d.qc_begin, a.V, a.ns)
-                                             : cm_query_token(row - d.qc_begin, a.S, a.V, a.ns, a.P);
+      // position heads: every query in cell-major order; token-wise heads: the special tokens,
+      // then (tensor-core plan) the patch queries in the cached order
+      const int r = row - d.qc_begin;
+      int tok;
+      if (d.kind != SAF3R_TOKEN) {
+        tok = cm_query_token(r, a.S, a.V, a.ns, a.P);
+      } else if (r < a.ns * a.S) {
+        tok = special_token(r, a.V, a.ns);
+      } else {
+        const int u = cache[a.tperm_off + (r - a.ns * a.S)];
+        if (u < 0 || u >= a.S * a.P) {
+          if (sub == 0) atomicCAS(err, 0, SAF3R_ERR_INDEX);
+          tok = a.ns;  // a patch token: the row is computed and never written
+        } else {
+          tok = (u / a.P) * a.V + a.ns + (u % a.P);
+        }
+      }
       const size_t src = (static_cast<size_t>(d.head) * a.N + tok) * kD;
       reinterpret_cast<uint4*>(qc + static_cast<size_t>(row) * kD)[sub] =
           reinterpret_cast<const uint4*>(q + src)[sub];

@@ -1376,7 +1376,7 @@ size_t rank_counts_bytes(int n_probe, int N) {
   return static_cast<size_t>(n_probe) * ((N + kRankChunk - 1) / kRankChunk) * 2 * sizeof(int);
 }
 
-size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows) {
+size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows, int tiles_P) {
   size_t b = 0;
   b += static_cast<size_t>(n_probe) * kProbePartials * kD * sizeof(double);
   b += static_cast<size_t>(n_probe) * kD * sizeof(float);
@@ -1392,6 +1392,8 @@ size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, lon
   if (corr) b += corr_ws(T, dim).end;
   b = ((b + 255) & ~size_t(255)) + 256;
   if (tok_rows > 0) b += token_ws(tok_rows, dim).end;
+  if (tok_rows > 0 && tiles_P > 0)
+    b = ((b + 255) & ~size_t(255)) + tok_tiles_workspace_bytes(static_cast<int>(tok_rows / tiles_P), tiles_P);
   return b;
 }
 
@@ -1550,7 +1552,7 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
   }
   if (sp.tok_kmax > 0) {
     // the token part of the workspace, after everything else
-    uint8_t* base = ws + select_workspace_bytes(sp.n_probe, sp.N, sp.T, sp.dim, sp.corr_kmax > 0, 0);
+    uint8_t* base = ws + select_workspace_bytes(sp.n_probe, sp.N, sp.T, sp.dim, sp.corr_kmax > 0, 0, 0);
     const long long R = static_cast<long long>(sp.S) * sp.P;
     const TokWs tw = token_ws(R, sp.dim);
     float* unit = reinterpret_cast<float*>(base + tw.unit);
@@ -1582,6 +1584,12 @@ cudaError_t launch_select(const SelectPlan& sp, const uint16_t* q, const uint16_
       token_rank_kernel<<<(rows + 7) / 8, 256, rsmem, stream>>>(scores, tw.ld, static_cast<int>(r0), rows, unit, sp.S,
                                                                 sp.P, sp.dim, sp.tok_kmax, cache + sp.tok_off);
       *n_launch += 2;
+    }
+    if (sp.tperm_off >= 0) {
+      // the patch query order and every group's unions and masks, after the lists
+      e = launch_tok_tiles(cache + sp.tok_off, sp.S, sp.P, sp.V, sp.ns, sp.tok_kmax, sp.tperm_off, sp.tg, sp.n_tg,
+                           cache, base + ((tw.end + 255) & ~size_t(255)), sp.err, stream, n_launch);
+      if (e != cudaSuccess) return e;
     }
   }
   return cudaGetLastError();

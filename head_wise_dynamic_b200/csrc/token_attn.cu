@@ -8,8 +8,9 @@
 // special-token query has no DINO feature and keeps every key: those rows are dense and run in
 // the tensor-core attention kernel.)
 //
-// No two patch query rows share a key set, so there is no dense block for the tensor cores: one
-// warp per query row, split into 8 groups of 4 lanes; a group takes kept keys n, n + 8 together
+// This kernel takes the patch queries of the token-wise heads that do not run in the tensor-core
+// kernel (a layout the union builder does not fit, or more plans than the plan array holds).
+// Each row walks its own keys: one warp per query row, split into 8 groups of 4 lanes; a group takes kept keys n, n + 8 together
 // (every 16th pair), each lane of it 16 of the 64 features (a 128-byte K row and V row gathered
 // from L2 by one group in one coalesced access each; both keys' K and V rows are requested
 // before any of them is used).  A group keeps its own running max, sum and accumulator in fp32;
@@ -109,10 +110,8 @@ __global__ void __launch_bounds__(256, 4) token_attn_kernel(const TokenAttnParam
     const int h = p.heads[hi], kf = p.k[hi];  // kf: per-frame budget of this head
     const Divider by_kf(static_cast<uint32_t>(kf)), by_ns(static_cast<uint32_t>(p.ns > 0 ? p.ns : 1));
     const size_t hb = static_cast<size_t>(h) * p.N * kD;
-    const int nl = p.S * kf;  // ranked keys; the special tokens follow, unless the tensor-core
-                              // kernel took them (then merged below)
-    const bool part = p.part_o[hi] != nullptr;
-    const int nk = part ? nl : nl + nsp;
+    const int nl = p.S * kf;  // ranked keys; the special tokens follow
+    const int nk = nl + nsp;
     const int32_t* lists = p.cache + p.tok_off + static_cast<size_t>(a) * p.S * p.tok_kmax;
     float qv[16];
     load16(p.q + hb + static_cast<size_t>(i) * kD + 16 * sub, qv);
@@ -179,20 +178,7 @@ __global__ void __launch_bounds__(256, 4) token_attn_kernel(const TokenAttnParam
         y0 = o[2 * g];
         y1 = o[2 * g + 1];
       }
-    float den = l;
-    if (part) {
-      // merge with the special keys' state: their output is normalised, its weight 2^lse
-      const float lse = p.part_lse[hi][a];
-      const float M = fmaxf(mm, lse);
-      const float fg = mm == -INFINITY ? 0.f : fast_exp2(mm - M);
-      const float fs = lse == -INFINITY ? 0.f : fast_exp2(lse - M);
-      const float2 ps =
-          *reinterpret_cast<const float2*>(p.part_o[hi] + static_cast<size_t>(a) * kD + 16 * sub + 2 * grp);
-      y0 = y0 * fg + ps.x * fs;
-      y1 = y1 * fg + ps.y * fs;
-      den = l * fg + fs;
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
     y0 *= inv;
     y1 *= inv;
     const size_t orow = hb + static_cast<size_t>(i) * kD + 16 * sub + 2 * grp;

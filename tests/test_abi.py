@@ -119,7 +119,8 @@ def test_token_cfg_validation():
 def test_token_select_workspace_on_host(S):
     """Token-wise heads add to the select workspace: fp32 and fp16 unit features of the R = S*P
     patch tokens and the fp16 scores of one chunk of query rows, at most 1 GiB of them (every
-    chunk a multiple of 128 rows, or all R rows)."""
+    chunk a multiple of 128 rows, or all R rows), and the query order's buckets (3P + 1 ints) and
+    sort keys (R 64-bit words)."""
     from saf3r_synth import Layout
     L = hw.layout_of(Layout(S=S, g=37 if S > 4 else 16, H=4))
     base = [HeadCfg(PROBE, k=64), HeadCfg(CORR, k=4), HeadCfg(SCAN, stride=4, phase=1), HeadCfg(SCAN, stride=8)]
@@ -130,8 +131,10 @@ def test_token_select_workspace_on_host(S):
     ld = (R + 7) // 8 * 8
     feats = R * L.dino_dim * 4 + R * ((L.dino_dim + 63) // 64 * 64) * 2
     chunk = min(R, max(128, (1 << 30) // (2 * ld) // 128 * 128))
-    assert w1 - w0 >= feats + chunk * ld * 2
-    assert w1 - w0 <= feats + min(R * ld * 2, (1 << 30)) + 4096
+    P = L.grid_h * L.grid_w
+    order = (3 * P + 1 + 63) // 64 * 64 * 4 + R * 8
+    assert w1 - w0 >= feats + chunk * ld * 2 + order
+    assert w1 - w0 <= feats + min(R * ld * 2, (1 << 30)) + order + 4096
 
 
 def test_baseline_stride_rule_in_the_library():

@@ -310,33 +310,56 @@ TOKEN_CASES = {
 }
 
 
-@pytest.mark.parametrize("which", ["probe", "tile", "token"])
+@pytest.mark.parametrize("which", ["probe", "tile", "token_order", "token_union"])
 def test_out_of_range_cached_index_is_reported(tiny, which):
-    """A cached index that points outside the layer (a probe key past N, a ranked tile past T, a
-    per-frame patch past P) is range-checked where it is consumed: the call records
-    SAF3R_ERR_INDEX, reads nothing out of range, and the next check finds the error word cleared.
-    The cache header's hash covers the layout and the configuration, not the lists, so the planted
-    value gets past the cache check."""
+    """A cached index that points outside the layer is range-checked where it is consumed: the
+    call records SAF3R_ERR_INDEX, reads nothing out of range, and the next check finds the error
+    word cleared.  Planted values: a probe key past N, a ranked tile past T, a token-wise patch
+    query past S*P in the cached query order, a token past N in an item's union.  The cache
+    header's hash covers the layout and the configuration, not the lists, so the planted value
+    gets past the cache check."""
     hw = _hw()
-    case = tiny if which != "token" else Case(TOKEN_CASES["token_mixed"])
+    case = tiny if which in ("probe", "tile") else Case(TOKEN_CASES["token_mixed"])
     heads = case.wl.heads
-    h, kind, bad = {"probe": (1, PROBE, case.L.N + 7), "tile": (2, CORR, case.L.T + 5),
-                    "token": (0, TOKEN, case.L.P + 3)}[which]
-    assert heads[h].kind == kind
+    L = case.L
     att, _ = run_gpu(case, heads)
-    lst = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).ravel().astype(np.int32)
     words = att.cache.view(torch.int32).cpu().numpy().copy()
-    starts = [i for i in np.flatnonzero(words[:len(words) - len(lst) + 1] == lst[0])
-              if np.array_equal(words[i:i + len(lst)], lst)]
-    assert len(starts) == 1, "the exported list is not one contiguous run of the cache"
-    words[starts[0] + len(lst) // 2] = bad
+
+    def find(lst):
+        starts = [i for i in np.flatnonzero(words[:len(words) - len(lst) + 1] == lst[0])
+                  if np.array_equal(words[i:i + len(lst)], lst)]
+        assert len(starts) == 1, "the exported list is not one contiguous run of the cache"
+        return starts[0]
+
+    if which in ("probe", "tile"):
+        h = 1 if which == "probe" else 2
+        assert heads[h].kind == (PROBE if which == "probe" else CORR)
+        lst = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h).ravel().astype(np.int32)
+        words[find(lst) + len(lst) // 2] = L.N + 7 if which == "probe" else L.T + 5
+    else:
+        # head 0 has the widest per-frame budget, so its lists are the cached block itself; the
+        # query order follows it (64-word aligned), then the first group's union lengths and unions
+        assert heads[0].kind == TOKEN and heads[0].k == max(hc.k for hc in heads if hc.kind == TOKEN)
+        lst = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, 0).ravel().astype(np.int32)
+        R = L.S * L.P
+        perm_at = (find(lst) + len(lst) + 63) // 64 * 64
+        assert np.array_equal(np.sort(words[perm_at:perm_at + R]), np.arange(R))  # a permutation
+        if which == "token_order":
+            words[perm_at + R // 2] = R + 3
+        else:
+            items = (R + 255) // 256
+            tn_at = (perm_at + R + 63) // 64 * 64
+            tu_at = (tn_at + items + 63) // 64 * 64
+            U0 = int(words[tn_at])
+            first = words[tu_at:tu_at + U0]
+            assert 0 < U0 and np.all(np.diff(first) > 0) and first[-1] < L.N  # item 0's union, ascending
+            words[tu_at + U0 // 2] = L.N + 11
     att.cache.copy_(torch.from_numpy(words).view(torch.uint8).to(att.cache.device))
     att(case.q, case.k, case.v)
     with pytest.raises(hw.Saf3rError) as e:
         hw.saf3r_check()
     assert e.value.status == hw.ERR_INDEX
     hw.saf3r_check()  # the error word was cleared
-
 
 def _check_token_heads(case, heads, att, sels, rows):
     """Per-frame lists of every token-wise head (the given query rows) against the oracle; each
