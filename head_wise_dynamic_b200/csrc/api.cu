@@ -96,19 +96,6 @@ bool make_map_3d(CUtensorMap* m, const void* base, long long rows, int H) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [rows][64] bf16 with a box of one row: the map of TMA row gathers (four rows per load)
-bool make_map_rows(CUtensorMap* m, const void* base, long long rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows < 1 ? 1 : rows)};
-  cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool make_map_2d(CUtensorMap* m, const void* base, long long rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
@@ -642,14 +629,14 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
   p.wait_budget = t_wait_budget;
   p.withhold_arrive = t_withhold_arrive ? 1 : 0;
   t_withhold_arrive = false;
+  p.k_rows = static_cast<const uint16_t*>(k);
+  p.v_rows = static_cast<const uint16_t*>(v);
   p.tok_perm = cl.tperm_off >= 0 && cache_i ? cache_i + cl.tperm_off : nullptr;
 
   if (t_ev_start && t_ev_stop && cudaEventRecord(t_ev_start, stream) != cudaSuccess) return SAF3R_ERR_CUDA;
   if (n_main > 0) {
-    CUtensorMap tq, tk, tv, tqc, tkc, tvc, tkg, tvg;
-    if (!make_map_3d(&tq, q, d.N, d.H) || !make_map_3d(&tk, k, d.N, d.H) || !make_map_3d(&tv, v, d.N, d.H) ||
-        !make_map_rows(&tkg, k, static_cast<long long>(d.H) * d.N) ||
-        !make_map_rows(&tvg, v, static_cast<long long>(d.H) * d.N))
+    CUtensorMap tq, tk, tv, tqc, tkc, tvc;
+    if (!make_map_3d(&tq, q, d.N, d.H) || !make_map_3d(&tk, k, d.N, d.H) || !make_map_3d(&tv, v, d.N, d.H))
       return SAF3R_ERR_CUDA;
     const void* kc_base = s.kc_rows > 0 ? static_cast<const void*>(kc) : k;
     const void* vc_base = s.kc_rows > 0 ? static_cast<const void*>(vc) : v;
@@ -658,7 +645,7 @@ saf3r_status run_attention(const saf3r_layout* L, const saf3r_head_cfg* cfg, con
         !make_map_2d(&tvc, vc_base, s.kc_rows > 0 ? s.kc_rows : 1) ||
         !make_map_2d(&tqc, qc_base, s.qc_rows > 0 ? s.qc_rows : 1))
       return SAF3R_ERR_CUDA;
-    st = cuda_status(launch_attention(p, tq, tk, tv, tqc, tkc, tvc, tkg, tvg, dev.sms, stream));
+    st = cuda_status(launch_attention(p, tq, tk, tv, tqc, tkc, tvc, dev.sms, stream));
     ++launches;
     if (st != SAF3R_OK) return st;
   }

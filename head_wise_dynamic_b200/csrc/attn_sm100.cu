@@ -16,16 +16,16 @@
 //
 // Token-wise heads' patch queries (q_src 4) come in a cached order that makes queries with the
 // same best matches neighbours; each item streams the head's special keys (derived rows) and then
-// the union of its rows' per-frame keys, whose K/V rows arrive by TMA row gathers (four listed
-// rows per instruction, 16 lanes of the producer warp), and every row keeps its own keys of that
+// the union of its rows' per-frame keys, whose scattered K and V rows the two otherwise idle warps
+// copy (cp.async, 16 bytes per lane, many rows in flight); every row keeps its own keys of that
 // union through a cached bitmask.
 //
 // Warp roles (12 warps, three warpgroups):
-//   warp 0      TMA producer: Q tiles, then K and V blocks into a 4-stage ring (for gathered
-//               runs 16 lanes issue the row gathers)
+//   warp 0      TMA producer: Q tiles, then K and V blocks into a 4-stage ring
 //   warp 1      MMA issuer: O_t += P_t V, then S_t = Q_t K^T of the next block (the whole warp
 //               waits and computes descriptors, one elected lane issues)
-//   warps 2-3   idle (their registers go to the softmax warpgroups)
+//   warps 2-3   token-wise items only: copy the union's K and V rows (cp.async), one key half each
+//               (most of their registers go to the softmax warpgroups)
 //   warps 4-11  softmax: warp w owns rows 32*(w%4)..+31 of a tile (the TMEM lanes it may
 //               read) and key half (w-4)/4 of every 128-key block; all eight warps work
 //               on tile 0, then on tile 1, so each tile's products run on the tensor
@@ -88,6 +88,8 @@ struct AttnSmem {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t vg_go[kStages];    // token-wise items: the producer found the stage free for the gather warps
+  uint64_t vg_done[kStages];  // token-wise items: both gather warps' K/V rows of the stage have landed
   Half info[kStages][2];      // the key halves of the block in each K/V stage (written by the producer)
   Seg segbuf[kSegBuf];        // the current item's key runs (copied by the producer warp, read by its lane 0)
   uint64_t pair[4];           // the two warps sharing rows 32*w..+31 (w = warp % 4) meet here at an item's end
@@ -241,50 +243,28 @@ __device__ __forceinline__ bool producer_item(const AttnParams& p, AttnSmem& sm,
   return true;
 }
 
-// Rows 4l..4l+3 of a gathered half (src 2) for lane l < 16, as rows of the [H*N][64] K/V maps.
-// Rows past the half's count, of an absent half, or whose listed token is out of range
-// (reported) load the head's token 0 instead: an in-range row whose keys every row masks.
-__device__ __forceinline__ int4 gather_rows(const AttnParams& p, const HeadPlan& hp, const Half& h, int lane) {
-  const int pad = hp.head * p.N;
-  int r[4] = {pad, pad, pad, pad};
-  const int b = 4 * lane;
-  if (lane < 16 && h.have && h.s.src == 2 && b < h.cnt) {
-    const int4 t4 = *reinterpret_cast<const int4*>(hp.glist + h.s.row0 + h.off + b);
-    const int t[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (b + i >= h.cnt) continue;
-      if (t[i] >= 0 && t[i] < p.N)
-        r[i] = hp.head * p.N + t[i];
-      else
-        atomicCAS(p.err, 0, SAF3R_ERR_INDEX);
-    }
-  }
-  return make_int4(r[0], r[1], r[2], r[3]);
-}
-
-// One 64-row half of a K or V stage: derived rows by one TMA box (lane 0), else (gathered rows,
-// or an absent half) four rows per lane of lanes 0-15 by TMA row gathers.
-__device__ __forceinline__ void load_half_gathered(const HeadPlan& hp, const Half& h, const int4& rows,
-                                                   uint8_t* dst, const CUtensorMap& m2, const CUtensorMap& mg,
-                                                   uint64_t* bar, int lane) {
-  if (h.have && h.s.src == 1) {
-    if (lane == 0) tma_load_2d(dst, &m2, 0, hp.kc_base + h.s.row0 + h.off, bar);
-  } else if (lane < 16) {
-    tma_gather4(dst + lane * 512, &mg, 0, rows.x, rows.y, rows.z, rows.w, bar);
-  }
-}
-
 // One item of a token-wise head's patch queries, run by the whole producer warp: derived Q rows
-// and the derived special K/V rows as TMA boxes, the union's K/V rows as TMA row gathers (each
-// full stage barrier expects one whole tile, as for the other heads).
+// and the derived special K/V rows as TMA boxes; the union's K and V rows come from the gather
+// warps (gather_role).  A stage's full barriers expect the bytes of its TMA halves and get this
+// warp's arrival once both gather warps report its rows landed (checked one block later).
 __device__ __forceinline__ bool producer_item_gather(const AttnParams& p, AttnSmem& sm, const CUtensorMap& tmQC,
-                                                     const CUtensorMap& tmKC, const CUtensorMap& tmVC,
-                                                     const CUtensorMap& tmKG, const CUtensorMap& tmVG,
-                                                     ItemInfo& it, const HeadPlan& hp, uint32_t& k_issued,
-                                                     uint32_t& v_issued, uint32_t& q_issued, int lane) {
+                                                     const CUtensorMap& tmKC, const CUtensorMap& tmVC, ItemInfo& it,
+                                                     const HeadPlan& hp, uint32_t& k_issued, uint32_t& v_issued,
+                                                     uint32_t& q_issued, uint32_t& vg_par, int lane) {
   volatile int* abort = &sm.abort;
   const long long budget = p.wait_budget;
+  int pend = -1;  // the stage waiting for the gather warps
+  auto release_v = [&]() -> bool {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.vg_done[pend], (vg_par >> pend) & 1u, abort, p.err,
+                                                      budget, SAF3R_ERR_TIMEOUT));
+    vg_par ^= 1u << pend;
+    if (lane == 0) {
+      mbar_arrive(&sm.k_full[pend]);
+      mbar_arrive(&sm.v_full[pend]);
+    }
+    pend = -1;
+    return ok;
+  };
   if (q_issued > 0 &&
       !__all_sync(0xffffffffu, mbar_wait(&sm.q_empty, (q_issued - 1) & 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)))
     return false;
@@ -298,31 +278,129 @@ __device__ __forceinline__ bool producer_item_gather(const AttnParams& p, AttnSm
   for (int b = 0; b < it.nblk; ++b) {
     const Half h0 = it.w.next();
     const Half h1 = it.w.next();
-    const int4 r0 = gather_rows(p, hp, h0, lane), r1 = gather_rows(p, hp, h1, lane);
     const uint32_t stage = k_issued % kStages, ph = (k_issued / kStages) & 1;
     if (k_issued >= kStages &&
         !__all_sync(0xffffffffu, mbar_wait(&sm.k_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)))
       return false;
-    if (lane == 0) mbar_arrive_expect_tx(&sm.k_full[stage], kTileBytes);
-    __syncwarp();
-    load_half_gathered(hp, h0, r0, sm.k[stage], tmKC, tmKG, &sm.k_full[stage], lane);
-    load_half_gathered(hp, h1, r1, sm.k[stage] + kHalfBytes, tmKC, tmKG, &sm.k_full[stage], lane);
+    if (lane == 0) {
+      const bool s0 = h0.have && h0.s.src == 1, s1 = h1.have && h1.s.src == 1;
+      if (s0 || s1) {
+        mbar_expect_tx(&sm.k_full[stage], (s0 ? kHalfBytes : 0) + (s1 ? kHalfBytes : 0));
+        if (s0) tma_load_2d(sm.k[stage], &tmKC, 0, hp.kc_base + h0.s.row0 + h0.off, &sm.k_full[stage]);
+        if (s1) tma_load_2d(sm.k[stage] + kHalfBytes, &tmKC, 0, hp.kc_base + h1.s.row0 + h1.off, &sm.k_full[stage]);
+      }
+    }
     ++k_issued;
     if (v_issued >= kStages &&
-        !__all_sync(0xffffffffu, mbar_wait(&sm.v_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT)))
+        !__all_sync(0xffffffffu, mbar_wait(&sm.v_empty[stage], ph ^ 1, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
+      if (pend >= 0) release_v();
       return false;
+    }
+    const bool t0 = h0.have && h0.s.src == 1, t1 = h1.have && h1.s.src == 1;
     if (lane == 0) {
-      // the block's halves for the softmax warps; the arrival below releases them with the stage
+      mbar_arrive(&sm.vg_go[stage]);  // the gather warps may fill this stage now
+      // the block's halves for the softmax warps; the arrival releases them with the stage
       sm.info[stage][0] = h0;
       sm.info[stage][1] = h1;
-      mbar_arrive_expect_tx(&sm.v_full[stage], kTileBytes);
+      if (t0 || t1) {
+        mbar_expect_tx(&sm.v_full[stage], (t0 ? kHalfBytes : 0) + (t1 ? kHalfBytes : 0));
+        if (t0) tma_load_2d(sm.v[stage], &tmVC, 0, hp.kc_base + h0.s.row0 + h0.off, &sm.v_full[stage]);
+        if (t1) tma_load_2d(sm.v[stage] + kHalfBytes, &tmVC, 0, hp.kc_base + h1.s.row0 + h1.off, &sm.v_full[stage]);
+      }
     }
-    __syncwarp();
-    load_half_gathered(hp, h0, r0, sm.v[stage], tmVC, tmVG, &sm.v_full[stage], lane);
-    load_half_gathered(hp, h1, r1, sm.v[stage] + kHalfBytes, tmVC, tmVG, &sm.v_full[stage], lane);
     ++v_issued;
+    if (pend >= 0 && !release_v()) {
+      pend = static_cast<int>(stage);
+      release_v();
+      return false;
+    }
+    pend = static_cast<int>(stage);
   }
-  return true;
+  return pend < 0 || release_v();
+}
+
+// Warps 2-3 on the items of token-wise heads' patch queries: warp 2 copies the union's K and V rows
+// of each block's first key half, warp 3 those of the second (cp.async, 16 bytes per lane, laid out
+// as a TMA box with 128-byte swizzle would be: chunk c of row r at chunk c ^ (r & 7); an absent
+// half, rows past its count and out-of-range tokens (reported) are zero), and each arrives on the
+// stage's vg_done once its rows have landed (checked one block later, so two blocks' copies are
+// in flight).  They start a block when the producer, which takes every block in order, reports
+// its stage free (vg_go): walking the other items' blocks themselves, they could otherwise run
+// phases ahead of the ring.  Other items are skipped; only the stage count advances.
+__device__ __forceinline__ void gather_role(const AttnParams& p, AttnSmem& sm, int kh, int lane) {
+  volatile int* abort = &sm.abort;
+  const long long budget = p.wait_budget;
+  const int col = lane & 7;
+  uint32_t kv = 0;      // key blocks of every item so far (the producer's count)
+  uint32_t go_par = 0;  // phase parity of each stage's vg_go
+  bool ok = true;
+  for (int item = blockIdx.x; ok && item < p.total_items; item += gridDim.x) {
+    ItemInfo it = item_info(p, item);
+    const HeadPlan& hp = p.heads[it.hi];
+    if (hp.q_src != 4) {
+      kv += it.nblk;
+      continue;
+    }
+    const uint16_t* vrows = p.v_rows + static_cast<size_t>(hp.head) * p.N * kD + col * 8;
+    const uint16_t* krows = p.k_rows + static_cast<size_t>(hp.head) * p.N * kD + col * 8;
+    int pend = -1;
+    for (int b = 0; b < it.nblk; ++b) {
+      const Half h0 = it.w.next();
+      const Half h1 = it.w.next();
+      const Half h = kh ? h1 : h0;
+      const bool copy = !(h.have && h.s.src == 1);
+      // listed tokens of this half: lane l holds rows l and l + 32 (-1: none)
+      int ta = -1, tb = -1;
+      if (copy && h.have) {
+        if (lane < h.cnt) ta = hp.glist[h.s.row0 + h.off + lane];
+        if (lane + 32 < h.cnt) tb = hp.glist[h.s.row0 + h.off + lane + 32];
+      }
+      const uint32_t stage = kv % kStages;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&sm.vg_go[stage], (go_par >> stage) & 1u, abort, p.err, budget, SAF3R_ERR_TIMEOUT))) {
+        ok = false;
+        break;
+      }
+      go_par ^= 1u << stage;
+      if (copy) {
+        const uint32_t base = smem_u32(sm.v[stage] + kh * kHalfBytes);
+        const uint32_t kbase = smem_u32(sm.k[stage] + kh * kHalfBytes);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = (lane >> 3) + 4 * i;
+          int t = __shfl_sync(0xffffffffu, i < 8 ? ta : tb, r & 31);
+          if (t >= p.N || t < -1) {
+            atomicCAS(p.err, 0, SAF3R_ERR_INDEX);
+            t = -1;
+          }
+          cp_async16(kbase + r * 128 + ((col ^ (r & 7)) << 4),
+                     t >= 0 ? static_cast<const void*>(krows + static_cast<size_t>(t) * kD)
+                            : static_cast<const void*>(p.v_rows),
+                     t >= 0 ? 16u : 0u);
+          cp_async16(base + r * 128 + ((col ^ (r & 7)) << 4),
+                     t >= 0 ? static_cast<const void*>(vrows + static_cast<size_t>(t) * kD)
+                            : static_cast<const void*>(p.v_rows),
+                     t >= 0 ? 16u : 0u);
+        }
+      }
+      cp_async_commit();
+      if (pend >= 0) {
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.vg_done[pend]);
+      }
+      pend = static_cast<int>(stage);
+      ++kv;
+    }
+    cp_async_wait<0>();
+    if (pend >= 0) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.vg_done[pend]);
+    }
+  }
+  cp_async_wait<0>();
 }
 
 // ------------------------------------------------------------------ TMA producer (one warp, lane 0 issues)
@@ -333,14 +411,14 @@ __device__ __forceinline__ bool producer_item_gather(const AttnParams& p, AttnSm
 __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm, const CUtensorMap& tmQ,
                                               const CUtensorMap& tmK, const CUtensorMap& tmV,
                                               const CUtensorMap& tmQC, const CUtensorMap& tmKC,
-                                              const CUtensorMap& tmVC, const CUtensorMap& tmKG,
-                                              const CUtensorMap& tmVG, int lane) {
+                                              const CUtensorMap& tmVC, int lane) {
   if (lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
   uint32_t k_issued = 0, v_issued = 0, q_issued = 0;
+  uint32_t vg_par = 0;  // phase parity of each stage's vg_done
   bool ok = true;
   for (int item = blockIdx.x; ok && item < p.total_items; item += gridDim.x) {
     ItemInfo it = item_info(p, item);
@@ -351,7 +429,7 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, AttnSmem& sm,
     }
     __syncwarp();
     if (hp.q_src == 4) {
-      ok = producer_item_gather(p, sm, tmQC, tmKC, tmVC, tmKG, tmVG, it, hp, k_issued, v_issued, q_issued, lane);
+      ok = producer_item_gather(p, sm, tmQC, tmKC, tmVC, it, hp, k_issued, v_issued, q_issued, vg_par, lane);
       __syncwarp();
     } else {
       if (lane == 0) ok = producer_item(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, it, hp, k_issued, v_issued, q_issued);
@@ -955,8 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmQC, const __grid_constant__ CUtensorMap tmKC,
-                      const __grid_constant__ CUtensorMap tmVC, const __grid_constant__ CUtensorMap tmKG,
-                      const __grid_constant__ CUtensorMap tmVG) {
+                      const __grid_constant__ CUtensorMap tmVC) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
@@ -979,6 +1056,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.o_done[t], 1);
     }
     for (int w = 0; w < 4; ++w) mbar_init(&sm.pair[w], 64);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.vg_go[s], 1);
+      mbar_init(&sm.vg_done[s], 2);
+    }
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -993,10 +1074,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) reg_dealloc_dec<104>();  // 104*128 + 200*256 = 168*384 registers
   if (warp == 0) {
-    producer_role(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, tmKG, tmVG, lane);
+    producer_role(p, sm, tmQ, tmK, tmV, tmQC, tmKC, tmVC, lane);
     __syncwarp();
   } else if (warp == 1) {
     mma_role(p, sm, tmem);
+    __syncwarp();
+  } else if (warp == 2 || warp == 3) {
+    gather_role(p, sm, warp - 2, lane);
     __syncwarp();
   } else if (warp >= 4) {
     reg_alloc_inc<200>();
@@ -1015,15 +1099,14 @@ size_t attn_smem_bytes() { return sizeof(AttnSmem) + 1024; }
 
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmQC, const CUtensorMap& tmKC,
-                             const CUtensorMap& tmVC, const CUtensorMap& tmKG, const CUtensorMap& tmVG,
-                             int num_sms, cudaStream_t stream) {
+                             const CUtensorMap& tmVC, int num_sms, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.total_items < num_sms ? p.total_items : num_sms;
   if (grid <= 0) return cudaSuccess;
-  attn_sm100_kernel<<<grid, kThreads, smem, stream>>>(p, tmQ, tmK, tmV, tmQC, tmKC, tmVC, tmKG, tmVG);
+  attn_sm100_kernel<<<grid, kThreads, smem, stream>>>(p, tmQ, tmK, tmV, tmQC, tmKC, tmVC);
   return cudaGetLastError();
 }
 

@@ -59,8 +59,7 @@ constexpr int kCacheHeaderBytes = 512;
 // A run of key rows of one head, fed to the attention kernel 64 rows at a time.
 // src 0: the caller's K/V ([H][N][64], row = token); src 1: the head's derived
 // rows in the workspace (row relative to the head's derived base); src 2: the tokens
-// listed at the head's gathered-key list (entry row0 + i, row0 a multiple of 4), rows gathered
-// from the caller's K/V.
+// listed at the head's gathered-key list (entry row0 + i), rows copied from the caller's K/V.
 struct Seg {
   int32_t src;
   int32_t row0;
@@ -129,6 +128,8 @@ struct AttnParams {
   const int* ok_flag;  // nonzero: cache check passed (NULL: no check)
   long long wait_budget;
   int32_t withhold_arrive;  // test hook: CTA 0's first softmax warp withholds its first P-ready arrival
+  const uint16_t* k_rows;   // the caller's K and V ([H][N][64] bf16): rows of gathered key runs
+  const uint16_t* v_rows;
   const int32_t* tok_perm;  // patch query order of the token-wise heads (in the cache)
   HeadPlan heads[kMaxHeads];
 };
@@ -221,8 +222,7 @@ saf3r_status validate_layout_cfg(const saf3r_layout* L, const saf3r_head_cfg* cf
 size_t attn_smem_bytes();
 cudaError_t launch_attention(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmQC, const CUtensorMap& tmKC,
-                             const CUtensorMap& tmVC, const CUtensorMap& tmKG, const CUtensorMap& tmVG,
-                             int num_sms, cudaStream_t stream);
+                             const CUtensorMap& tmVC, int num_sms, cudaStream_t stream);
 size_t select_workspace_bytes(int n_probe, int N, int T, int dim, bool corr, long long tok_rows, int tiles_P);
 size_t token_rank_smem_bytes(int P, int kmax);
 size_t token_sim_smem_bytes();
