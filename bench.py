@@ -40,8 +40,8 @@ L2_NOTE = "inputs larger than L2 (Q/K/V 3 x 281 MB per call)"
 # (dram__bytes_read.sum + dram__bytes_write.sum of one S=100-view layer call, one launch, a
 # 1-pass metric set; its summary is kept under profiles/), valid only for the kernel source it was
 # taken on: a changed kernel reports null until it is re-captured.
-ATTN_TRAFFIC = {"kernel_source_sha256": "d3c1155f587330ec4575c56cf8226458a4a428c12aa5a8c567c2b320dbc5c298",
-                "bytes_per_launch": 606443008 + 265179136, "workload": "s100"}
+ATTN_TRAFFIC = {"kernel_source_sha256": "070ee568bbd2f24b66132f561c1773dcdf52e9fffacc3ec5e108d2a7d2c3fca6",
+                "bytes_per_launch": 598363648 + 265262080, "workload": "s100"}
 
 
 def kernel_source_sha256():
