@@ -94,7 +94,14 @@ enum { SAF3R_OP_SELECT = 0, SAF3R_OP_SPARSE = 1, SAF3R_OP_DENSE = 2, SAF3R_OP_PR
  * and, if any head is CORR or HYBRID, the ranked key-tile list of every query
  * tile (int32 [T][kmax], best first; T = ceil(N/64), kmax = largest such k),
  * and, if any head is TOKEN, the ranked per-frame lists of every patch query
- * (int32 [S*P][S][kmax] patch indices, best first; kmax = largest TOKEN k).
+ * (int32 [S*P][S][kmax] patch indices, best first; kmax = largest TOKEN k),
+ * and, where the layout allows (S*P patches, P up to about 6,000, at most
+ * 2^28 union entries per budget), the patch queries' order for the tensor
+ * cores plus, per distinct TOKEN k and per 256 queries of that order, room
+ * for the union of their kept tokens (S * min(256 k, P) entries, int32) and
+ * one 64-bit mask per query and 64 union entries: about
+ * 36 * ceil(S*P/256) * S * min(256 k, P) bytes per distinct k (2.6 GB at
+ * S = 100, P = 1369, k = 16).
  * Returns 0 for an invalid layout or cfg.
  */
 size_t saf3r_cache_bytes(const saf3r_layout* layout, const saf3r_head_cfg* cfg);
@@ -132,6 +139,11 @@ size_t saf3r_profile_workspace_bytes(const saf3r_layout* layout, const saf3r_hea
  *     exactly (fp64), so the ranking is that of the fp64 cosines rounded to
  *     fp32.  The workspace then holds the fp16 scores of up to 1 GiB of query
  *     rows at a time.  Needs dino_dim <= 384 (SAF3R_ERR_UNSUPPORTED otherwise).
+ *     The patch queries are then ordered by their best match in frame 0,
+ *     then in frame 1 (queries that see the same scene point become
+ *     neighbours), and every 256 queries of that order get the ascending
+ *     union of their kept tokens and a per-query bitmask over it, which the
+ *     attention streams through the tensor cores.
  *   - POSITION, SCAN and DENSE heads need no cached state (a HYBRID head's
  *     lattice neither).
  * q, k: bf16 [H][N][d]; dino: fp32 patch features, or NULL when no head is

@@ -361,6 +361,61 @@ def test_out_of_range_cached_index_is_reported(tiny, which):
     assert e.value.status == hw.ERR_INDEX
     hw.saf3r_check()  # the error word was cleared
 
+def test_token_unions_are_exactly_their_rows_keys():
+    """The token-wise structures of a built cache, checked exactly on the host against the cached
+    per-frame lists: the patch query order is a permutation of the S*P patch queries; for every
+    budget k (one group per distinct k, in head order) and every 256 queries of the order, the union
+    is the ascending set of tokens those queries keep (their first k list entries of every frame),
+    and query r's mask bit for union entry e is set exactly when r keeps that token (rows past the
+    last query keep nothing).  Placement: after the lists, each region starts on a 64-word boundary:
+    the order, then per group the union lengths, the unions (ucap = S*min(256k, P) rounded up to 64
+    entries per item) and the masks ([ucap/64][256] 64-bit words per item)."""
+    hw = _hw()
+    case = Case(TOKEN_CASES["token_mixed"])
+    heads = case.wl.heads
+    L = case.L
+    att, _ = run_gpu(case, heads)
+    words = att.cache.view(torch.int32).cpu().numpy()
+    ks = []
+    for hc in heads:
+        if hc.kind == TOKEN and hc.k not in ks:
+            ks.append(hc.k)
+    kmax = max(ks)
+    h0 = [i for i, hc in enumerate(heads) if hc.kind == TOKEN and hc.k == kmax][0]
+    lst = hw.saf3r_cache_export(att.layout, att.cfg, att.cache, h0).ravel().astype(np.int32)
+    at = [i for i in np.flatnonzero(words[:len(words) - len(lst) + 1] == lst[0])
+          if np.array_equal(words[i:i + len(lst)], lst)]
+    assert len(at) == 1
+    R, S, P, V, ns = L.S * L.P, L.S, L.P, L.V, L.n_special
+    lists = lst.reshape(R, S, kmax)
+    al = lambda x: (x + 63) // 64 * 64
+    perm_at = al(at[0] + len(lst))
+    perm = words[perm_at:perm_at + R]
+    assert np.array_equal(np.sort(perm), np.arange(R))
+    items = (R + 255) // 256
+    off = perm_at + R
+    for k in ks:
+        ucap = al(S * min(256 * k, P))
+        tn_at = al(off)
+        tu_at = al(tn_at + items)
+        tm_at = al(tu_at + items * ucap)
+        off = tm_at + items * (ucap // 64) * 256 * 2
+        masks = words[tm_at:off].view(np.uint64).reshape(items, ucap // 64, 256)
+        for m in range(items):
+            rows = perm[m * 256:(m + 1) * 256]
+            keep = [set().union(*[set((f * V + ns + lists[u, f, :k]).tolist()) for f in range(S)]) for u in rows]
+            union = np.array(sorted(set().union(*keep)), dtype=np.int64)
+            U = int(words[tn_at + m])
+            assert U == len(union), (k, m)
+            assert np.array_equal(words[tu_at + m * ucap:tu_at + m * ucap + U], union), (k, m)
+            bits = (masks[m][np.arange(U) // 64] >> (np.arange(U) % 64).astype(np.uint64)[:, None]) & np.uint64(1)
+            want = np.zeros((U, 256), bool)
+            pos = {t: e for e, t in enumerate(union.tolist())}
+            for r, ks_r in enumerate(keep):
+                want[[pos[t] for t in ks_r], r] = True
+            assert np.array_equal(bits.astype(bool), want), (k, m)
+
+
 def _check_token_heads(case, heads, att, sels, rows):
     """Per-frame lists of every token-wise head (the given query rows) against the oracle; each
     head is added to `sels`.  Returns {head: lists identical}."""
