@@ -175,3 +175,32 @@ def test_profile_rejects_a_token_candidate_without_dino():
     p = 0x1000
     assert lib.saf3r_profile_heads(ctypes.byref(L), cand, 2, p, p, p, None, 0.01, chosen, nmse, pairs, p,
                                    None) == hw.ERR_INVALID
+
+
+@pytest.mark.parametrize("S,g,on", [(4, 16, True), (200, 37, False)])
+def test_token_cache_bytes_follow_the_documented_placement(S, g, on):
+    """The cache size of a layer with token-wise heads, added up from the documented placement:
+    header, probe lists, ranked tile lists and their order, the per-frame lists, then (when the
+    unions fit: at most 2^28 union entries per budget) the patch query order and, per distinct k,
+    union lengths, unions and masks, each region on a 64-word boundary.  S=200 at 37x37 patches
+    and k=16 needs 2.9e8 union entries: no unions (the gather kernel takes those heads)."""
+    from saf3r_synth import Layout
+    heads = [HeadCfg(TOKEN, k=16), HeadCfg(CORR, k=4), HeadCfg(TOKEN, k=5), HeadCfg(PROBE, k=100)]
+    lay = Layout(S=S, g=g, H=4)
+    L = hw.layout_of(lay)
+    al = lambda x: (x + 63) // 64 * 64
+    ints = 512 // 4 + al(100)                      # header, the probe head's list
+    ints += lay.T * 4 + lay.T                      # ranked tiles (kmax 4), their grouping order
+    ints = al(ints) + lay.S * lay.P * lay.S * 16   # per-frame lists, tok_kmax 16
+    R = lay.S * lay.P
+    items = (R + 255) // 256
+    if on:
+        ints = al(ints) + R
+        for k in (16, 5):
+            ucap = al(lay.S * min(256 * k, lay.P))
+            ints = al(ints) + items
+            ints = al(ints) + items * ucap
+            ints = al(ints) + items * (ucap // 64) * 256 * 2
+    else:
+        assert items * al(lay.S * min(256 * 5, lay.P)) > (1 << 28)
+    assert hw.saf3r_cache_bytes(L, hw.cfg_array(heads)) == (ints * 4 + 255) // 256 * 256
