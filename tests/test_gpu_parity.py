@@ -307,6 +307,12 @@ TOKEN_CASES = {
     # token-wise heads mixed with the other kinds in one call
     "token_mixed": _custom(4, 16, [HeadCfg(TOKEN, k=16), HeadCfg(CORR, k=4), HeadCfg(TOKEN, k=5),
                                    HeadCfg(POSITION)], D=256),
+    # no special tokens: every item's keys are its union alone
+    "token_no_specials": _custom(3, 10, [HeadCfg(TOKEN, k=6), HeadCfg(SCAN, stride=3, phase=1),
+                                         HeadCfg(TOKEN, k=2), HeadCfg(PROBE, k=30)], ns=0),
+    # one view: the query order has no second frame; k = P keeps the whole view
+    "token_one_view": _custom(1, 12, [HeadCfg(TOKEN, k=7), HeadCfg(TOKEN, k=144), HeadCfg(CORR, k=2),
+                                      HeadCfg(POSITION)]),
 }
 
 
