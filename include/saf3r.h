@@ -185,6 +185,12 @@ saf3r_status saf3r_select_kv_static(const saf3r_layout* layout, const saf3r_head
  * on the device through the cache header hash; a mismatch records
  * SAF3R_ERR_INVALID and leaves `out` unwritten).  q, k, v may be fresh
  * tensors of a later layer call: the cached sets are reused as they are.
+ * All heads run in one tensor-core launch; a TOKEN head's patch queries run
+ * there over their cached per-256-query key unions (each query masked to its
+ * own keys) when the layout has unions and the launch's per-head plans fit
+ * (at most 64 plans: one per head, plus one per TOKEN head with special
+ * tokens), else in a per-query gather kernel.  Both give the exact softmax
+ * over each query's kept keys.
  * out: bf16 [H][N][d] (out_is_fp32 = 0) or fp32 (out_is_fp32 = 1).
  * workspace: saf3r_workspace_bytes(layout, cfg, SAF3R_OP_SPARSE) bytes.
  */
