@@ -474,11 +474,11 @@ def test_token_heads_tied_features(n_feat):
     check_rows(case, heads, sels, out, lambda h: np.arange(L.N))
 
 
-def test_token_heads_with_and_without_a_partial_plan():
+def test_token_heads_with_and_without_a_tensor_core_plan():
     """62 heads, 6 of them token-wise: the tensor-core kernel's plan array (64) holds the 62 heads'
-    plans and the partial plans of only the first 2 token heads, so those 2 take their patch queries'
-    special keys on the tensor cores and merge, while the other 4 take them in the gather kernel.
-    Every row of every head against the oracle."""
+    plans and the patch-query plans of only the first 2 token heads, so those 2 run their patch
+    queries on the tensor cores over the cached unions while the other 4 run them in the gather
+    kernel.  Every row of every head against the oracle."""
     heads = [HeadCfg(SCAN, stride=4, phase=h % 4) for h in range(56)] + \
             [HeadCfg(TOKEN, k=4), HeadCfg(TOKEN, k=9)] * 3
     case = Case(_custom(4, 10, heads, seed=95))
