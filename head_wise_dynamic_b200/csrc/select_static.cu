@@ -59,7 +59,8 @@ extern "C" saf3r_status saf3r_select_kv_static(const saf3r_layout* layout, const
   void* scratch = nullptr;
   const saf3r_status st = scratch_address(&scratch);
   if (st != SAF3R_OK) return st;
-  // Everything the build reads from the scratch it first writes in the same call (the
-  // grouping bitsets, the only part that must start at zero, are cleared by the call itself).
+  // Everything the build reads from the scratch it first writes in the same call (the parts
+  // that must start at zero - the probe ranking's counters, the grouping bitsets and the
+  // token-wise ordering's buckets - are cleared by the call itself).
   return saf3r_select_kv(layout, cfg, q, k, dino, cache, scratch, stream);
 }
